@@ -1,0 +1,48 @@
+"""I12: the chunk algebra the prefill kernel is built on reproduces the token recurrence.
+
+The fp64 chunk model (tests/chunk_model.py) must agree with the oracle to ~1e-12 for any
+chunk and sub-block size, with ragged tails, a nonzero initial state and the worst-case
+decay g = -5 on every channel (where unfactored exponents over a 64-token chunk would
+overflow).  With bf16 operands emulated at the kernel's rounding points it must stay well
+inside the 2e-2 bf16 tolerance.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from chunk_model import chunk_forward
+from helpers import max_rel_err, random_problem
+
+
+@pytest.mark.parametrize("C,sub", [(64, 32), (64, 16), (32, 16), (16, 16)])
+@pytest.mark.parametrize("worst_decay", [False, True])
+def test_chunk_form_matches_oracle(C, sub, worst_decay):
+    rng = np.random.default_rng(7)
+    q, k, v, g, beta, S0 = random_problem(rng, 1, 150, 2, 16, 12)
+    if worst_decay:
+        g = np.full_like(g, -5.0)
+    o_ref, ST_ref = oracle.forward(q, k, v, g, beta, S0, nthreads=2)
+    o, ST = chunk_forward(q, k, v, g, beta, S0, C=C, sub=sub)
+    assert max_rel_err(o, o_ref) < 1e-11, max_rel_err(o, o_ref)
+    assert max_rel_err(ST, ST_ref) < 1e-11, max_rel_err(ST, ST_ref)
+
+
+def test_chunk_form_slow_decay_with_state():
+    rng = np.random.default_rng(8)
+    q, k, v, g, beta, S0 = random_problem(rng, 1, 200, 1, 32, 32)
+    g = g * 0.02                                    # nearly no forgetting: the state carries far
+    o_ref, ST_ref = oracle.forward(q, k, v, g, beta, S0, nthreads=2)
+    o, ST = chunk_forward(q, k, v, g, beta, S0, C=64, sub=32)
+    assert max_rel_err(o, o_ref) < 1e-11 and max_rel_err(ST, ST_ref) < 1e-11
+
+
+@pytest.mark.parametrize("zg_mean", [0.0, -2.0, -6.0])
+def test_bf16_operands_stay_inside_tolerance(zg_mean):
+    rng = np.random.default_rng(9)
+    q, k, v, g, beta, S0 = random_problem(rng, 1, 320, 1, 64, 64)
+    g = -5.0 / (1.0 + np.exp(-(rng.standard_normal(g.shape) + zg_mean)))
+    o_ref, ST_ref = oracle.forward(q, k, v, g, beta, S0, nthreads=2)
+    o, ST = chunk_forward(q, k, v, g, beta, S0, C=64, sub=32, bf16=True)
+    # half the 2e-2 bf16 tolerance, before the final bf16 rounding of o
+    assert max_rel_err(o, o_ref) < 1e-2, max_rel_err(o, o_ref)
+    assert max_rel_err(ST, ST_ref) < 1e-2, max_rel_err(ST, ST_ref)
