@@ -1,0 +1,359 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA hot path on B200: chunked prefill + decode step, one JSON line.
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+  * prefill: kda_forward_chunked over the K3-shaped workload B=4, T=8192, H=96,
+    dk=dv=128, bf16 inputs, fp32 state (S0 ~ N(0, 0.02^2), decay logits z ~ N(-2, 1));
+  * decode: one kda_decode_step over 256 sequences x 96 heads of 128x128 fp32 states,
+    updated in place (fresh bf16 token each step, from a ring of pre-drawn inputs).
+`value` is prefill tokens/s (B*T per prefill / device time of the prefill launches,
+summed over ranks for N > 1: weak scaling, every rank runs its own batch, no collective
+on the data path).  Decode states/s, the roofline of each kernel, the end-to-end figure
+through the public API with host buffers, the oracle's CPU baseline and the clocks seen
+during the timed region are reported in the same line.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s (K3 shape, H=96, d=128) and decode states/s; % of roofline"
+PREFILL = dict(name="k3_b4_t8k", B=4, T=8192, H=96, dk=128, dv=128, dtype="bf16", s0_std=0.02, zg_mean=-2.0)
+DECODE = dict(name="decode_b256_h96", batch=256, H=96, dk=128, dv=128, dtype="bf16")
+DECODE_RING = 8
+
+
+def prefill_alg_bytes(B, T, H, dk, dv, elem=2, with_s0=True, with_st=True):
+    """Algorithmic HBM bytes of one prefill launch: every input read once, every output written once."""
+    per_token_head = elem * (3 * dk + dv) + elem + elem * dv   # q, k, g, v, beta in; o out
+    per_head = 4 * dk * dv * (int(with_s0) + int(with_st))        # S0 in, S_T out (fp32)
+    return B * T * H * per_token_head + B * H * per_head
+
+
+def decode_alg_bytes(batch, H, dk, dv, elem=2):
+    """Per step: the fp32 state read and written once, plus the token's inputs and o."""
+    return batch * H * (2 * 4 * dk * dv + elem * (3 * dk + dv) + elem + elem * dv)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_attention_recurrence_forward_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_tag):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current sources."""
+    prof = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(prof):
+        return None
+    sha = kernel_source_sha()
+    for name in sorted(os.listdir(prof)):
+        if not name.endswith(".md"):
+            continue
+        text = open(os.path.join(prof, name)).read()
+        m = re.search(r"traffic_record:\s*kernel=(\S+)\s+sources=(\S+)\s+dram_bytes_per_launch=(\d+)", text)
+        if m and m.group(1) == kernel_tag and m.group(2) == sha:
+            return int(m.group(3))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"kda_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1])); maxes.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": max(maxes) if maxes else None,
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+def oracle_baseline(budget_s=15.0, seed=0):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the prefill workload.
+
+    The sample is n_heads full-length heads of the K3 workload (T = 8192, d = 128); the
+    result is scaled to the metric's unit: tokens/s = (token-heads/s) / H.
+    """
+    import torch
+    import oracle
+    from linear_attention_recurrence_forward_b200.inputs import make_prefill_inputs
+    cores = len(os.sched_getaffinity(0))
+    T, H, d = PREFILL["T"], PREFILL["H"], PREFILL["dk"]
+    # calibrate on one short head
+    cal = make_prefill_inputs(1, 512, 1, d, d, "bf16", seed=seed + 1, zg_mean=PREFILL["zg_mean"])
+    t0 = time.perf_counter()
+    oracle.forward(*cal[:5], None, nthreads=1)
+    per_token_head = (time.perf_counter() - t0) / 512
+    n_heads = max(cores, int(budget_s * cores / (per_token_head * T)))
+    n_heads = max(cores, (n_heads // cores) * cores)
+    n_heads = min(n_heads, 4 * 96)
+    q, k, v, g, beta, S0 = make_prefill_inputs(1, T, n_heads, d, d, "bf16", seed=seed, s0_std=0.02,
+                                               zg_mean=PREFILL["zg_mean"])
+    t0 = time.perf_counter()
+    oracle.forward(q, k, v, g, beta, S0, nthreads=cores)
+    dt = time.perf_counter() - t0
+    token_heads_per_s = n_heads * T / dt
+    return {"value": token_heads_per_s / H, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n_heads} heads x {T} tokens of the K3 prefill workload (d=128), fp64, {dt:.1f} s; "
+                      f"tokens/s = token-heads/s / {H}",
+            "seconds": dt, "token_heads_per_s": token_heads_per_s}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    per_step = []
+    base = None
+    for i in range(args.warmup + args.steps):
+        r = oracle_baseline(budget_s=8.0, seed=i)
+        if i >= args.warmup:
+            per_step.append(r)
+        base = r
+    value = statistics.mean(r["value"] for r in per_step)
+    secs = statistics.mean(r["seconds"] for r in per_step)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": PREFILL["name"], "B": PREFILL["B"], "T": PREFILL["T"], "H": PREFILL["H"],
+                       "dk": PREFILL["dk"], "dv": PREFILL["dv"]},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": base["cores"], "kind": "oracle",
+                             "sample": base["sample"]},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import linear_attention_recurrence_forward_b200 as kda
+    from linear_attention_recurrence_forward_b200.inputs import make_prefill_inputs, make_decode_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+
+    P = PREFILL
+    q, k, v, g, beta, S0 = make_prefill_inputs(P["B"], P["T"], P["H"], P["dk"], P["dv"], P["dtype"],
+                                               seed=1000 + rank, s0_std=P["s0_std"], zg_mean=P["zg_mean"],
+                                               device=str(dev))
+    o = torch.empty((P["B"], P["T"], P["H"], P["dv"]), dtype=q.dtype, device=dev)
+    ST = torch.empty((P["B"], P["H"], P["dk"], P["dv"]), dtype=torch.float32, device=dev)
+    D = DECODE
+    gen = torch.Generator(device=str(dev))
+    gen.manual_seed(2000 + rank)
+    ring = [make_decode_inputs(D["batch"], D["H"], D["dk"], D["dv"], D["dtype"], gen=gen, device=str(dev))
+            for _ in range(DECODE_RING)]
+    S = torch.zeros((D["batch"], D["H"], D["dk"], D["dv"]), dtype=torch.float32, device=dev)
+    od = torch.empty((D["batch"], D["H"], D["dv"]), dtype=q.dtype, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        kda.kda_forward_chunked(q, k, v, g, beta, S0, o=o, S_T=ST, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        x = ring[i % DECODE_RING]
+        kda.kda_decode_step(*x, S, o=od, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    status = kda.kda_get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after warm-up: {kda.kda_status_string(status)}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    sampler = ClockSampler(visible.split(",")[local_rank].strip() if visible else str(local_rank))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    status = kda.kda_get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status after timing: {kda.kda_status_string(status)}")
+
+    total_ms = t_start.elapsed_time(t_end)
+    prefill_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    decode_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    tm = torch.tensor([total_ms, sum(prefill_ms), sum(decode_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+    total_ms, prefill_sum, decode_sum = tm.tolist()
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
+    host_in = [t.to("cpu").pin_memory() for t in (q, k, v, g, beta)]
+    host_s0 = S0.to("cpu").pin_memory()
+    host_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    e2e_steps = max(1, min(args.steps, 3))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        dq, dk_, dv_, dg, db = (t.to(dev, non_blocking=True) for t in host_in)
+        ds0 = host_s0.to(dev, non_blocking=True)
+        oo, _ = kda.kda_forward_chunked(dq, dk_, dv_, dg, db, ds0, stream=stream)
+        host_o.copy_(oo, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    h2d = sum(t.numel() * t.element_size() for t in host_in) + host_s0.numel() * 4
+    d2h = host_o.numel() * host_o.element_size()
+
+    tokens_per_prefill = P["B"] * P["T"]
+    value = world * tokens_per_prefill * args.steps / (prefill_sum / 1e3)
+    states = D["batch"] * D["H"]
+    decode_states_per_s = world * states * args.steps / (decode_sum / 1e3)
+    peak, peak_kind = measured_peaks()
+    pb = prefill_alg_bytes(P["B"], P["T"], P["H"], P["dk"], P["dv"])
+    prefill_launch_ms = prefill_sum / args.steps
+    achieved = pb / (prefill_launch_ms / 1e3) / 1e9
+    db_ = decode_alg_bytes(D["batch"], D["H"], D["dk"], D["dv"])
+    decode_launch_ms = decode_sum / args.steps
+    dec_achieved = db_ / (decode_launch_ms / 1e3) / 1e9
+    impl_tag = "prefill_tc" if kda.lib().kda_forward_chunked_impl(None, None, None, None, None, None, None,
+                                                                    None, 1, 0, 1, 128, 128, 0, 1, None) == 0 \
+        else "prefill_simt"
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_baseline(budget_s=args.cpu_budget)
+        cpu = {k_: cpu[k_] for k_ in ("value", "unit", "cores", "kind", "sample")}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{P['name']} prefill + {D['name']} decode step",
+                   "B": P["B"], "T": P["T"], "H": P["H"], "dk": P["dk"], "dv": P["dv"],
+                   "decode_batch": D["batch"], "l2": "inputs larger than L2 (4.1 GB prefill, 1.6 GB decode state)",
+                   "parallelism": f"replicas x{world} (independent batches, no collective)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": recorded_traffic(impl_tag),
+                     "kernel": impl_tag, "alg_bytes_per_launch": pb, "launch_ms": prefill_launch_ms,
+                     "peak_kind": peak_kind},
+        "decode": {"states_per_s": decode_states_per_s, "tokens_per_s": decode_states_per_s / D["H"],
+                   "ms_per_step": decode_launch_ms,
+                   "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peak, "unit": "GB/s",
+                                "frac": dec_achieved / peak, "alg_bytes_per_launch": db_,
+                                "traffic": recorded_traffic("decode")}},
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * tokens_per_prefill / (e2e_ms.item() / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "prefill through kda_forward_chunked with pinned host inputs copied in and o copied out"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

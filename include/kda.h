@@ -1,0 +1,141 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention (KDA) recurrence library.
+ *
+ * KDA is a gated delta-rule linear attention with a per-channel forget gate.  Per
+ * batch element b and head h it carries a state S in R^{dk x dv} and, for each token t,
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(exp g_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * i.e. decay every row i of the state by exp(g_t[i]), let the decayed memory predict v_t
+ * from k_t, write only the residual (scaled by beta_t) back along k_t, then read the
+ * updated state with q_t.  Sources:
+ *   - "Day 21" course page (ai.air7.fun/decks/k3-course-30/day-21): interview item D19
+ *     (fixed-size d x d state, delta-rule residual update, per-channel decay gate),
+ *     quiz Q8 (state built from k^T v products, O(1) memory), quiz Q9 (predict with the
+ *     old memory, overwrite with the residual v - S k only);
+ *   - Kimi K3 skill card (skillsmp.com), quick facts: the log-decay is a lower-bounded
+ *     scaled sigmoid with g_min = -5, which keeps the diagonal tiles of the chunked form
+ *     dense enough for tensor-core products;
+ *   - podcast show-notes (scripod.com), section 2.1: chunk-recurrent form (RetNet) and
+ *     gated delta rule (Gated DeltaNet), which this library's prefill follows.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library never
+ *     allocates, frees or retains caller memory.  It owns one small static device status
+ *     word per device (see kda_get_device_status).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream).  A return of KDA_OK means the work was validated and enqueued.
+ *   - Tensors are contiguous, row-major, with the layouts stated per function.
+ *   - `dtype` applies to q, k, v, g, beta and o.  The state is always fp32.
+ *   - g is the per-channel LOG-decay itself (g <= 0; the gate nonlinearity is the
+ *     caller's).  There is no query scaling and no q/k normalisation inside the library.
+ *   - Supported sizes: dk, dv in {64, 128}; B, H >= 1; T >= 0 (T == 0 copies S0 to S_T).
+ *     Every pointer must be 16-byte aligned.
+ *   - Errors: argument checks happen before anything is enqueued and return a negative
+ *     kda_status; a failed launch returns KDA_ERR_CUDA.  A device-side wait that runs
+ *     out (it never hangs) sets the device status word to KDA_ERR_TIMEOUT, which
+ *     kda_get_device_status reports.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* == cudaStream_t's pointee; keeps this header free of CUDA includes */
+
+/* Exported symbols (the library is built with hidden visibility by default). */
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = -1, /* null pointer, non-positive size, aliasing that is not allowed */
+    KDA_ERR_UNSUPPORTED = -2, /* dtype or head size the library has no kernel for */
+    KDA_ERR_MISALIGNED = -3,  /* a pointer is not 16-byte aligned */
+    KDA_ERR_CUDA = -4,        /* a CUDA runtime/driver call failed (launch, attribute, ...) */
+    KDA_ERR_TIMEOUT = -5      /* a device-side bounded wait gave up (reported by the status word) */
+} kda_status;
+
+typedef enum { KDA_DTYPE_BF16 = 0, KDA_DTYPE_FP32 = 1 } kda_dtype;
+
+/* Prefill kernel selection for kda_forward_chunked_impl. */
+typedef enum {
+    KDA_IMPL_AUTO = 0,    /* tcgen05 kernel when it supports the shape, else the SIMT kernel */
+    KDA_IMPL_TCGEN05 = 1, /* chunkwise tensor-core kernel: bf16, dk = dv = 128 only */
+    KDA_IMPL_SIMT = 2     /* fp32 CUDA-core kernel: every supported dtype and size */
+} kda_impl;
+
+/*
+ * kda_forward_chunked -- prefill: run the recurrence over T tokens for every (b, h).
+ *
+ * Computes o_t for t = 1..T and the final state S_T, starting from S0 (the chunkwise
+ * parallel form with 64-token chunks; exact up to rounding, see the header comment).
+ *
+ *   q, k, g : [B, T, H, dk]   dtype     (g = log-decay, per channel)
+ *   v       : [B, T, H, dv]   dtype
+ *   beta    : [B, T, H]       dtype     (write strength, one scalar per token and head)
+ *   S0      : [B, H, dk, dv]  fp32, or NULL for a zero initial state
+ *   o       : [B, T, H, dv]   dtype     output (bf16 outputs are rounded to nearest even)
+ *   S_T     : [B, H, dk, dv]  fp32, or NULL when the final state is not wanted.
+ *             S_T may alias S0 exactly (in-place state carry); any other overlap
+ *             between outputs and inputs is not allowed.
+ *   dtype   : kda_dtype.
+ *
+ * Returns KDA_OK, or a negative kda_status (nothing is enqueued on error).
+ */
+KDA_API int kda_forward_chunked(const void* q, const void* k, const void* v, const void* g,
+                        const void* beta, const float* S0, void* o, float* S_T, int B, int T,
+                        int H, int dk, int dv, int dtype, struct CUstream_st* stream);
+
+/*
+ * kda_forward_chunked_impl -- kda_forward_chunked with an explicit kernel choice
+ * (kda_impl).  Same arguments, layouts and semantics; returns KDA_ERR_UNSUPPORTED when
+ * the requested kernel does not cover the dtype/shape.
+ */
+KDA_API int kda_forward_chunked_impl(const void* q, const void* k, const void* v, const void* g,
+                             const void* beta, const float* S0, void* o, float* S_T, int B,
+                             int T, int H, int dk, int dv, int dtype, int impl,
+                             struct CUstream_st* stream);
+
+/*
+ * kda_decode_step -- one token for every (b, h), state updated in place.
+ *
+ * Same recurrence with T = 1 (the memory-bound state read-modify-write of decoding):
+ *   S <- Diag(exp g) S;  u = beta (v - S^T k);  S <- S + k u^T;  o = S^T q.
+ *
+ *   q, k, g : [B, H, dk]      dtype
+ *   v       : [B, H, dv]      dtype
+ *   beta    : [B, H]          dtype
+ *   S       : [B, H, dk, dv]  fp32, read and written in place (must not be NULL)
+ *   o       : [B, H, dv]      dtype output
+ *
+ * Returns KDA_OK or a negative kda_status (nothing is enqueued on error).
+ */
+KDA_API int kda_decode_step(const void* q, const void* k, const void* v, const void* g,
+                    const void* beta, float* S, void* o, int B, int H, int dk, int dv,
+                    int dtype, struct CUstream_st* stream);
+
+/*
+ * kda_get_device_status -- synchronise `stream`, then return and clear the status word
+ * of the current device: KDA_OK, KDA_ERR_TIMEOUT (a kernel's bounded wait gave up; its
+ * outputs are then undefined), or KDA_ERR_CUDA if the synchronisation itself failed.
+ */
+KDA_API int kda_get_device_status(struct CUstream_st* stream);
+
+/* kda_status_string -- static, human-readable name of a kda_status value. */
+KDA_API const char* kda_status_string(int status);
+
+/* kda_version -- library version as major*10000 + minor*100 + patch. */
+KDA_API int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,170 @@
+"""Python binding of the B200 KDA recurrence library (ctypes over the C ABI in include/kda.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA kernels of
+libkda_b200.so.  There is no CPU fallback; if the library is missing or a call fails,
+these functions raise.
+
+    from linear_attention_recurrence_forward_b200 import kda_forward_chunked, kda_decode_step
+    o, S_T = kda_forward_chunked(q, k, v, g, beta, S0)        # prefill, torch CUDA tensors
+    o = kda_decode_step(q, k, v, g, beta, S)                   # one token, S updated in place
+
+Layouts (contiguous): q, k, g [B, T, H, dk]; v, o [B, T, H, dv]; beta [B, T, H];
+states [B, H, dk, dv] fp32.  Decode drops the T axis.  dtype: bf16 or fp32 (all of q, k,
+v, g, beta share it; o gets it too).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "kda_forward_chunked",
+    "kda_decode_step",
+    "kda_get_device_status",
+    "kda_status_string",
+    "KdaError",
+    "lib",
+    "LIB_PATH",
+    "STATUS",
+    "IMPL",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda_b200.so")
+
+STATUS = {
+    "KDA_OK": 0,
+    "KDA_ERR_INVALID_ARG": -1,
+    "KDA_ERR_UNSUPPORTED": -2,
+    "KDA_ERR_MISALIGNED": -3,
+    "KDA_ERR_CUDA": -4,
+    "KDA_ERR_TIMEOUT": -5,
+}
+DTYPE = {torch.bfloat16: 0, torch.float32: 1}
+IMPL = {"auto": 0, "tcgen05": 1, "simt": 2}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+class KdaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {kda_status_string(status)} ({status})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it first (python -m linear_attention_recurrence_forward_b200.build "
+                "or __graft_entry__.build()); there is no fallback implementation")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I = ctypes.c_void_p, ctypes.c_int
+        L.kda_forward_chunked.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P]
+        L.kda_forward_chunked.restype = I
+        L.kda_forward_chunked_impl.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P]
+        L.kda_forward_chunked_impl.restype = I
+        L.kda_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P]
+        L.kda_decode_step.restype = I
+        L.kda_get_device_status.argtypes = [P]
+        L.kda_get_device_status.restype = I
+        L.kda_status_string.argtypes = [I]
+        L.kda_status_string.restype = ctypes.c_char_p
+        L.kda_version.argtypes = []
+        L.kda_version.restype = I
+        _lib = L
+    return _lib
+
+
+def kda_status_string(status: int) -> str:
+    return lib().kda_status_string(int(status)).decode()
+
+
+def _stream_handle(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream or None
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _check(t: torch.Tensor, name: str, shape, dtype, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def kda_forward_chunked(q, k, v, g, beta, S0=None, *, o=None, S_T=None, return_state: bool = True,
+                        impl: str = "auto", stream=None):
+    """Prefill over [B, T, H, *] CUDA tensors.  Returns (o, S_T) (S_T None if not requested).
+
+    S_T may be passed in (and may be S0 itself for an in-place state carry).
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    if dt not in DTYPE:
+        raise ValueError(f"unsupported dtype {dt}")
+    for name, t, shape in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("v", v, (B, T, H, dv)),
+                           ("g", g, (B, T, H, dk)), ("beta", beta, (B, T, H))):
+        _check(t, name, shape, dt, dev)
+    if S0 is not None:
+        _check(S0, "S0", (B, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    else:
+        _check(o, "o", (B, T, H, dv), dt, dev)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    elif S_T is not None:
+        _check(S_T, "S_T", (B, H, dk, dv), torch.float32, dev)
+    with torch.cuda.device(dev):
+        rc = lib().kda_forward_chunked_impl(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                                            _ptr(o), _ptr(S_T), B, T, H, dk, dv, DTYPE[dt], IMPL[impl],
+                                            _stream_handle(stream))
+    if rc != 0:
+        raise KdaError("kda_forward_chunked", rc)
+    return o, S_T
+
+
+def kda_decode_step(q, k, v, g, beta, S, *, o=None, stream=None):
+    """One token for every (b, h).  q, k, g [B, H, dk]; v [B, H, dv]; beta [B, H]; S updated in place."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    if dt not in DTYPE:
+        raise ValueError(f"unsupported dtype {dt}")
+    for name, t, shape in (("q", q, (B, H, dk)), ("k", k, (B, H, dk)), ("v", v, (B, H, dv)),
+                           ("g", g, (B, H, dk)), ("beta", beta, (B, H))):
+        _check(t, name, shape, dt, dev)
+    _check(S, "S", (B, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=dt, device=dev)
+    else:
+        _check(o, "o", (B, H, dv), dt, dev)
+    with torch.cuda.device(dev):
+        rc = lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                                   B, H, dk, dv, DTYPE[dt], _stream_handle(stream))
+    if rc != 0:
+        raise KdaError("kda_decode_step", rc)
+    return o
+
+
+def kda_get_device_status(stream=None, device=None) -> int:
+    """Synchronise the stream, then return and clear the device status word (0 = OK)."""
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        return int(lib().kda_get_device_status(_stream_handle(stream)))

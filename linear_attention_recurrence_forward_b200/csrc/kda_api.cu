@@ -1,0 +1,179 @@
+// C ABI of the KDA library: argument validation, kernel choice, the device status word.
+//
+// Everything here runs on the host before a launch; nothing is enqueued unless every
+// check passes.  The kernels themselves live in kda_decode.cu, kda_prefill_simt.cu and
+// kda_prefill_tc.cu.
+#include <mutex>
+#include <stdint.h>
+
+#include "kda_internal.cuh"
+
+// One status word per device (this module is loaded once per device context).  Kernels
+// receive its device address as an argument and set it on a timed-out wait.
+__device__ int g_kda_status_word = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mutex;
+int* g_status_addr[kMaxDevices] = {nullptr};
+
+int* status_word_for_current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_status_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_kda_status_word) != cudaSuccess) return nullptr;
+        g_status_addr[dev] = static_cast<int*>(p);
+    }
+    return g_status_addr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool head_dim_ok(int d) { return d == 64 || d == 128; }
+
+struct Range {
+    uintptr_t lo, hi;  // [lo, hi)
+};
+Range range_of(const void* p, size_t bytes) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return Range{a, a + bytes};
+}
+bool overlaps(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.lo != a.hi && b.lo != b.hi; }
+
+size_t elem_size(int dtype) { return dtype == KDA_DTYPE_BF16 ? 2 : 4; }
+
+int validate_prefill(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                     const float* S0, const void* o, const float* ST, int B, int T, int H, int dk,
+                     int dv, int dtype) {
+    if (B <= 0 || H <= 0 || T < 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_FP32) return KDA_ERR_UNSUPPORTED;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    // 64-bit element counts must stay far from overflow
+    const double elems = (double)B * (double)T * (double)H * (double)(dk > dv ? dk : dv);
+    if (elems > 9.0e15) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, g, beta, S0, o, ST};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    if (T > 0) {
+        const size_t es = elem_size(dtype);
+        const size_t n_tok = (size_t)B * T * H;
+        const Range ro = range_of(o, n_tok * dv * es);
+        const Range ins[] = {range_of(q, n_tok * dk * es), range_of(k, n_tok * dk * es),
+                             range_of(v, n_tok * dv * es), range_of(g, n_tok * dk * es),
+                             range_of(beta, n_tok * es)};
+        for (const Range& r : ins)
+            if (overlaps(ro, r)) return KDA_ERR_INVALID_ARG;
+        const size_t sbytes = (size_t)B * H * dk * dv * sizeof(float);
+        if (S0 && overlaps(ro, range_of(S0, sbytes))) return KDA_ERR_INVALID_ARG;
+        if (ST) {
+            const Range rs = range_of(ST, sbytes);
+            if (overlaps(rs, ro)) return KDA_ERR_INVALID_ARG;
+            for (const Range& r : ins)
+                if (overlaps(rs, r)) return KDA_ERR_INVALID_ARG;
+        }
+    }
+    if (S0 && ST && S0 != ST) {
+        const size_t sbytes = (size_t)B * H * dk * dv * sizeof(float);
+        if (overlaps(range_of(S0, sbytes), range_of(ST, sbytes))) return KDA_ERR_INVALID_ARG;
+    }
+    return KDA_OK;
+}
+
+int forward_impl(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                 const float* S0, void* o, float* ST, int B, int T, int H, int dk, int dv, int dtype,
+                 int impl, cudaStream_t stream) {
+    if (impl != KDA_IMPL_AUTO && impl != KDA_IMPL_TCGEN05 && impl != KDA_IMPL_SIMT)
+        return KDA_ERR_INVALID_ARG;
+    int rc = validate_prefill(q, k, v, g, beta, S0, o, ST, B, T, H, dk, dv, dtype);
+    if (rc != KDA_OK) return rc;
+    kda::PrefillArgs a{q, k, v, g, beta, S0, o, ST, B, T, H, dk, dv, dtype, nullptr};
+    const bool tc_ok = kda::prefill_tc_supports(a);
+    if (impl == KDA_IMPL_TCGEN05 && !tc_ok) return KDA_ERR_UNSUPPORTED;
+    if (T == 0) {
+        // No tokens: the final state is the initial state.
+        if (!ST) return KDA_OK;
+        const size_t sbytes = (size_t)B * H * dk * dv * sizeof(float);
+        cudaError_t e = S0 ? (S0 == ST ? cudaSuccess
+                                       : cudaMemcpyAsync(ST, S0, sbytes, cudaMemcpyDeviceToDevice, stream))
+                           : cudaMemsetAsync(ST, 0, sbytes, stream);
+        return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
+    a.status = status_word_for_current_device();
+    if (!a.status) return KDA_ERR_CUDA;
+    cudaError_t e;
+    if (impl == KDA_IMPL_SIMT || (impl == KDA_IMPL_AUTO && !tc_ok)) e = kda::launch_prefill_simt(a, stream);
+    else e = kda::launch_prefill_tc(a, stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_forward_chunked(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                        const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv,
+                        int dtype, struct CUstream_st* stream) {
+    return forward_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, dtype, KDA_IMPL_AUTO, stream);
+}
+
+int kda_forward_chunked_impl(const void* q, const void* k, const void* v, const void* g,
+                             const void* beta, const float* S0, void* o, float* S_T, int B, int T,
+                             int H, int dk, int dv, int dtype, int impl, struct CUstream_st* stream) {
+    return forward_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, dtype, impl, stream);
+}
+
+int kda_decode_step(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                    float* S, void* o, int B, int H, int dk, int dv, int dtype,
+                    struct CUstream_st* stream) {
+    if (B <= 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_FP32) return KDA_ERR_UNSUPPORTED;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !g || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
+    if ((double)B * (double)H > 2.0e9) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, g, beta, S, o};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+    const size_t es = elem_size(dtype);
+    const size_t n = (size_t)B * H;
+    const Range rs = range_of(S, n * dk * dv * sizeof(float));
+    const Range ro = range_of(o, n * dv * es);
+    const Range ins[] = {range_of(q, n * dk * es), range_of(k, n * dk * es), range_of(v, n * dv * es),
+                         range_of(g, n * dk * es), range_of(beta, n * es)};
+    if (overlaps(rs, ro)) return KDA_ERR_INVALID_ARG;
+    for (const Range& r : ins)
+        if (overlaps(rs, r) || overlaps(ro, r)) return KDA_ERR_INVALID_ARG;
+    kda::DecodeArgs a{q, k, v, g, beta, S, o, B, H, dk, dv, dtype, status_word_for_current_device()};
+    if (!a.status) return KDA_ERR_CUDA;
+    return kda::launch_decode(a, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_get_device_status(struct CUstream_st* stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
+    int* addr = status_word_for_current_device();
+    if (!addr) return KDA_ERR_CUDA;
+    int value = 0;
+    if (cudaMemcpy(&value, addr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpy(addr, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return KDA_ERR_CUDA;
+    return value;
+}
+
+const char* kda_status_string(int status) {
+    switch (status) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+        case KDA_ERR_MISALIGNED: return "KDA_ERR_MISALIGNED";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+        default: return "KDA_ERR_UNKNOWN";
+    }
+}
+
+int kda_version(void) { return 100; }
+
+}  // extern "C"

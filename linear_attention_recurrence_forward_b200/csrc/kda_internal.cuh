@@ -1,0 +1,61 @@
+// Internal declarations shared by the library's translation units (not installed).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+// Arguments of one prefill launch, already validated by the C ABI layer.
+struct PrefillArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const void* g;
+    const void* beta;
+    const float* S0;  // may be null (zero state)
+    void* o;
+    float* ST;        // may be null
+    int B, T, H, dk, dv;
+    int dtype;        // kda_dtype
+    int* status;      // device status word
+};
+
+struct DecodeArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const void* g;
+    const void* beta;
+    float* S;
+    void* o;
+    int B, H, dk, dv;
+    int dtype;
+    int* status;
+};
+
+// Launchers: return cudaSuccess or the launch error.  Defined in their kernel's .cu file.
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
+bool prefill_tc_supports(const PrefillArgs& a);
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
+
+// Element loads/stores for the two input dtypes.
+__device__ __forceinline__ float load_elem(const float* p, size_t i) { return p[i]; }
+__device__ __forceinline__ float load_elem(const __nv_bfloat16* p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void store_elem(float* p, size_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void store_elem(__nv_bfloat16* p, size_t i, float x) {
+    p[i] = __float2bfloat16_rn(x);
+}
+
+// Set the device status word once (first error wins).
+__device__ __forceinline__ void report_status(int* status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+}  // namespace kda

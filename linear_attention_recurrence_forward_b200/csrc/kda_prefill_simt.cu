@@ -1,0 +1,160 @@
+// KDA prefill on CUDA cores in fp32, token by token (every dtype, dk/dv in {64, 128}).
+//
+// This is the library's fp32 path (the bf16 tensor-core kernel cannot reach fp32
+// accuracy) and the fallback kernel for head sizes the tensor-core kernel does not
+// cover.  It runs the recurrence exactly as defined, one token at a time:
+//   S <- Diag(exp g_t) S;  u = beta_t (v_t - S^T k_t);  S <- S + k_t u^T;  o_t = S^T q_t
+// ("Day 21" course page, interview item D19 and quiz Q9), with fp32 arithmetic and the
+// state held in registers for the whole sequence.
+//
+// The recurrence is separable over the dv columns of S (column c only ever mixes with
+// v[c] and u[c]), so each CTA owns one (b, h) and a 32-column slice of the state: more
+// CTAs for the same problem, and 16 state values per thread.
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kSimtThreads = 256;
+constexpr int kSlice = 32;                 // state columns per CTA
+constexpr int kLpr = kSlice / 4;           // threads per row (float4 each) = 8
+constexpr int kRpp = kSimtThreads / kLpr;  // rows per pass = 32
+
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(kSimtThreads)
+kda_prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+                        const Tin* __restrict__ g, const Tin* __restrict__ beta,
+                        const float* S0, Tin* __restrict__ o, float* ST, int T, int H) {
+    constexpr int RPT = DK / kRpp;  // rows per thread (4 or 2)
+    constexpr int NW = kSimtThreads / 32;
+    constexpr int NSLICE = DV / kSlice;
+
+    __shared__ float qs[2][DK], ks[2][DK], es[2][DK], vs[2][kSlice], bs[2];
+    __shared__ float4 red_a[NW][kLpr], red_b[NW][kLpr];
+    __shared__ float4 us[kLpr];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int c4 = tid % kLpr, rg = tid / kLpr;
+    const int slice = blockIdx.x % NSLICE;
+    const size_t bh = blockIdx.x / NSLICE;
+    const int b = (int)(bh / H), h = (int)(bh % H);
+    const int col0 = slice * kSlice;
+
+    float4 s[RPT];
+#pragma unroll
+    for (int j = 0; j < RPT; ++j) {
+        const int r = rg + j * kRpp;
+        if (S0) s[j] = *reinterpret_cast<const float4*>(S0 + (bh * DK + r) * DV + col0 + 4 * c4);
+        else s[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+
+    auto stage = [&](int t, int buf) {
+        const size_t row = ((size_t)b * T + t) * H + h;
+        if (tid < DK) {
+            qs[buf][tid] = load_elem(q, row * DK + tid);
+            ks[buf][tid] = load_elem(k, row * DK + tid);
+            es[buf][tid] = expf(load_elem(g, row * DK + tid));
+        } else if (tid < DK + kSlice) {
+            vs[buf][tid - DK] = load_elem(v, row * DV + col0 + (tid - DK));
+        } else if (tid == DK + kSlice) {
+            bs[buf] = load_elem(beta, row);
+        }
+    };
+
+    if (T > 0) stage(0, 0);
+    __syncthreads();
+    for (int t = 0; t < T; ++t) {
+        const int buf = t & 1;
+        // decay, then the partial column sums S'^T k and S'^T q over this thread's rows
+        float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+            const int r = rg + j * kRpp;
+            const float e = es[buf][r], kr = ks[buf][r], qr = qs[buf][r];
+            s[j].x *= e; s[j].y *= e; s[j].z *= e; s[j].w *= e;
+            pa.x += s[j].x * kr; pa.y += s[j].y * kr; pa.z += s[j].z * kr; pa.w += s[j].w * kr;
+            pb.x += s[j].x * qr; pb.y += s[j].y * qr; pb.z += s[j].z * qr; pb.w += s[j].w * qr;
+        }
+#pragma unroll
+        for (int off = kLpr; off < 32; off <<= 1) {
+            pa.x += __shfl_xor_sync(0xffffffffu, pa.x, off); pa.y += __shfl_xor_sync(0xffffffffu, pa.y, off);
+            pa.z += __shfl_xor_sync(0xffffffffu, pa.z, off); pa.w += __shfl_xor_sync(0xffffffffu, pa.w, off);
+            pb.x += __shfl_xor_sync(0xffffffffu, pb.x, off); pb.y += __shfl_xor_sync(0xffffffffu, pb.y, off);
+            pb.z += __shfl_xor_sync(0xffffffffu, pb.z, off); pb.w += __shfl_xor_sync(0xffffffffu, pb.w, off);
+        }
+        if (lane < kLpr) { red_a[warp][lane] = pa; red_b[warp][lane] = pb; }
+        __syncthreads();
+        // Every thread is past iteration t-1 here, so the other buffer is free: stage the
+        // next token into it (read only after the second barrier below).
+        if (t + 1 < T) stage(t + 1, buf ^ 1);
+        if (warp == 0) {
+            float kq = 0.f;
+#pragma unroll
+            for (int i = lane; i < DK; i += 32) kq += ks[buf][i] * qs[buf][i];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+            if (lane < kLpr) {
+                float4 a = red_a[0][lane], bb = red_b[0][lane];
+#pragma unroll
+                for (int w = 1; w < NW; ++w) {
+                    const float4 ta = red_a[w][lane], tb = red_b[w][lane];
+                    a.x += ta.x; a.y += ta.y; a.z += ta.z; a.w += ta.w;
+                    bb.x += tb.x; bb.y += tb.y; bb.z += tb.z; bb.w += tb.w;
+                }
+                const float bt = bs[buf];
+                float4 u;
+                u.x = bt * (vs[buf][4 * lane + 0] - a.x);
+                u.y = bt * (vs[buf][4 * lane + 1] - a.y);
+                u.z = bt * (vs[buf][4 * lane + 2] - a.z);
+                u.w = bt * (vs[buf][4 * lane + 3] - a.w);
+                us[lane] = u;
+                const size_t oo = (((size_t)b * T + t) * H + h) * DV + col0 + 4 * lane;
+                store_elem(o, oo + 0, bb.x + kq * u.x);
+                store_elem(o, oo + 1, bb.y + kq * u.y);
+                store_elem(o, oo + 2, bb.z + kq * u.z);
+                store_elem(o, oo + 3, bb.w + kq * u.w);
+            }
+        }
+        __syncthreads();
+        const float4 u = us[c4];
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+            const float kr = ks[buf][rg + j * kRpp];
+            s[j].x += kr * u.x; s[j].y += kr * u.y; s[j].z += kr * u.z; s[j].w += kr * u.w;
+        }
+    }
+    if (ST) {
+#pragma unroll
+        for (int j = 0; j < RPT; ++j) {
+            const int r = rg + j * kRpp;
+            *reinterpret_cast<float4*>(ST + (bh * DK + r) * DV + col0 + 4 * c4) = s[j];
+        }
+    }
+}
+
+template <typename Tin, int DK, int DV>
+cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s) {
+    const unsigned grid = (unsigned)((size_t)a.B * a.H * (DV / kSlice));
+    kda_prefill_simt_kernel<Tin, DK, DV><<<grid, kSimtThreads, 0, s>>>(
+        static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
+        static_cast<const Tin*>(a.g), static_cast<const Tin*>(a.beta), a.S0, static_cast<Tin*>(a.o),
+        a.ST, a.T, a.H);
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t dispatch_dims(const PrefillArgs& a, cudaStream_t s) {
+    if (a.dk == 128 && a.dv == 128) return launch_t<Tin, 128, 128>(a, s);
+    if (a.dk == 128 && a.dv == 64) return launch_t<Tin, 128, 64>(a, s);
+    if (a.dk == 64 && a.dv == 128) return launch_t<Tin, 64, 128>(a, s);
+    return launch_t<Tin, 64, 64>(a, s);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s) {
+    if (a.dtype == KDA_DTYPE_BF16) return dispatch_dims<__nv_bfloat16>(a, s);
+    return dispatch_dims<float>(a, s);
+}
+
+}  // namespace kda
