@@ -1,7 +1,660 @@
-// Placeholder for the tcgen05 chunkwise prefill kernel (not yet built).
+// KDA chunked prefill on sm_100a: TMA loads, tcgen05 tensor-core products with TMEM
+// accumulators, fp32 state carried across 64-token chunks.  bf16 inputs, dk = dv = 128.
+//
+// Method (chunk-recurrent form of the gated delta rule: podcast show-notes section 2.1,
+// RetNet chunk recurrence + Gated DeltaNet gated delta rule; delta rule of the "Day 21"
+// course page, quiz Q9).  For one head and a chunk of C = 64 tokens with local index r,
+// state S (dk x dv) at the chunk start, Gam_r = sum_{t<=r} g_t (per channel):
+//
+//   Kt_r = k_r e^{Gam_r},  Qt_r = q_r e^{Gam_r},  Kb_j = k_j e^{Gam_C - Gam_j}
+//   A_rj = beta_r sum_i k_r[i] k_j[i] e^{Gam_r[i]-Gam_j[i]}   (j < r)
+//   P_rj =        sum_i q_r[i] k_j[i] e^{Gam_r[i]-Gam_j[i]}   (j <= r)
+//   T = (I + A)^{-1} Diag(beta)           (the WY / UT transform of the delta rule)
+//   U = T (V - Kt S)                       (the delta-rule residuals of the chunk)
+//   O = Qt S + P U
+//   S <- Diag(e^{Gam_C}) S + Kb^T U
+//
+// This is an exact rewrite of the token recurrence.  The pair factors e^{Gam_r-Gam_j}
+// are formed from two per-token factors against a reference token b (e^{Gam_r-Gam_b}
+// e^{Gam_b-Gam_j}).  The chunk is split into two 32-token blocks: the off-diagonal block
+// uses b = 31 (both factors <= 1), each diagonal block its middle token (16 or 48), where
+// each factor is at most e^{5*16} = e^{80} < FLT_MAX because the log-decay is bounded
+// below by -5 (the skill card's quick facts: the bounded scaled-sigmoid gate is what lets
+// the diagonal tiles run as dense tensor-core matmuls).
+//
+// Per CTA: one (b, h), the whole chunk sequence.  Tensor-core products per chunk:
+//   MMA1 [Qt0;Kt0;Qt1;Kt1](mid refs) x [Kh0;Kh1]^T    -> diagonal blocks of P and A
+//   MMA2 [Qt1;Kt1](ref 31)            x Kh0^T         -> off-diagonal block
+//   MMA3 [Kt;Qt] x S_bf16                             -> Kt S (Y = V - Kt S) and Qt S
+//   MMA4 T x Y                                        -> U
+//   MMA5 P x U   (accumulated onto Qt S)              -> O
+//   MMA6 Kb^T x U (accumulated onto the decayed fp32 state in TMEM) -> new S
+// The 64x64 triangular solve runs in fp32 on the CUDA cores.  Every M = 64 product is
+// issued as M = 128 with the unused 64 rows reading other (valid) shared memory, so all
+// accumulators use the one-row-per-lane TMEM layout; those lanes are never read.
+#include <cudaTypedefs.h>
+#include <mutex>
+
 #include "kda_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace kda {
-bool prefill_tc_supports(const PrefillArgs&) { return false; }
-cudaError_t launch_prefill_tc(const PrefillArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+using namespace sm100;
+
+constexpr int kC = 64;         // chunk length
+constexpr int kD = 128;        // dk = dv
+constexpr int kThreads = 256;  // 8 warps
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // bounded waits: 2 s
+
+// ---- shared memory map (bytes from a 1024-aligned base) ----
+constexpr uint32_t OFF_RAW_Q = 0;          // TMA destination, bf16 [64 tok][128], 2 boxes of 8 KB
+constexpr uint32_t OFF_RAW_K = 16384;
+constexpr uint32_t OFF_RAW_G = 32768;
+constexpr uint32_t OFF_RAW_V = 49152;
+constexpr uint32_t OFF_AP = 65536;         // operands of MMA1/2, reused after they complete
+constexpr uint32_t OFF_A1 = OFF_AP;                 // K-major, 128 rows, 2 atoms x 16 KB
+constexpr uint32_t OFF_B1 = OFF_AP + 32768;         // K-major, 64 rows, 2 atoms x 8 KB
+constexpr uint32_t OFF_A2 = OFF_AP + 49152;         // rows 64..127 only, 2 atoms x 8 KB
+constexpr uint32_t OFF_B2 = OFF_AP + 65536;         // K-major, 32 rows, 2 atoms x 4 KB
+constexpr uint32_t OFF_T = OFF_AP;                  // after MMA1/2: T rows 0..63 (K = 64)
+constexpr uint32_t OFF_PV = OFF_AP + 16384;         //   P as rows 64..127 of a tile starting here
+constexpr uint32_t OFF_KBAR = OFF_AP + 32768;       //   Kb, MN-major A (M = dk), 2 atoms x 8 KB
+constexpr uint32_t OFF_AF = OFF_AP + 49152;         //   A (fp32 64x64) for the solve
+constexpr uint32_t OFF_KQ = OFF_AP + 73728;         // [Kt; Qt], K-major, 128 rows, 2 atoms x 16 KB
+constexpr uint32_t OFF_SB = OFF_KQ + 32768;         // S in bf16, MN-major B (K = dk), 2 atoms x 16 KB
+constexpr uint32_t OFF_YU = OFF_SB + 32768;         // Y then U, MN-major B (K = 64), 2 atoms x 8 KB
+constexpr uint32_t SMEM_BYTES = OFF_YU + 16384;     // 221184
+constexpr uint32_t OFF_X = OFF_RAW_Q;               // solve: X = (I+A)^-1, fp32 64x64 (raw q is dead)
+constexpr uint32_t OFF_W = OFF_RAW_K;               // solve scratch, fp32 3 x 16x16
+constexpr uint32_t SMEM_DYN = SMEM_BYTES + 1024;    // + alignment slack
+
+// ---- TMEM columns (fp32 accumulators, 128 lanes) ----
+constexpr uint32_t TM_S = 0;     // S (dk lanes x dv columns), fp32 master state
+constexpr uint32_t TM_C = 128;   // MMA3 result: lanes 0-63 Kt S, lanes 64-127 Qt S (+ P U = O)
+constexpr uint32_t TM_U = 256;   // MMA4 result: lanes 0-63 U
+constexpr uint32_t TM_AP = 384;  // MMA1 (64 cols) and MMA2 (32 cols)
+constexpr uint32_t TM_COLS = 512;
+
+constexpr uint32_t ID_MMA1 = idesc_bf16_f32(128, 64, false, false);
+constexpr uint32_t ID_MMA2 = idesc_bf16_f32(128, 32, false, false);
+constexpr uint32_t ID_KxMN = idesc_bf16_f32(128, 128, false, true);
+constexpr uint32_t ID_MNxMN = idesc_bf16_f32(128, 128, true, true);
+
+struct TcParams {
+    const __nv_bfloat16* beta;
+    const float* S0;
+    __nv_bfloat16* o;
+    float* ST;
+    int* status;
+    int B, T, H;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&p);
+}
+__device__ __forceinline__ float bf16_at(const uint8_t* base, uint32_t off) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
+}
+__device__ __forceinline__ void put_bf16(uint8_t* base, uint32_t off, float x) {
+    *reinterpret_cast<__nv_bfloat16*>(base + off) = __float2bfloat16_rn(x);
+}
+
+// Issue one K-major-A / any-B product of K = 16*ksteps.  a_atom / b_atom: byte distance
+// between 64-column K atoms of a K-major operand; b_mn: B is MN-major (then b_lbo is the
+// distance between its 64-wide N atoms and each K step advances 16 rows = 2048 B).
+__device__ __forceinline__ void issue_mma(uint32_t d_tmem, uint32_t a_base, uint32_t a_atom, bool a_mn,
+                                          uint32_t a_lbo, uint32_t b_base, uint32_t b_atom, bool b_mn,
+                                          uint32_t b_lbo, int ksteps, uint32_t idesc, bool accumulate) {
+#pragma unroll 1
+    for (int kk = 0; kk < ksteps; ++kk) {
+        const uint32_t a = a_mn ? a_base + kk * 2048u : a_base + (kk >> 2) * a_atom + (kk & 3) * 32u;
+        const uint32_t b = b_mn ? b_base + kk * 2048u : b_base + (kk >> 2) * b_atom + (kk & 3) * 32u;
+        mma_bf16(d_tmem, smem_desc_sw128(a, a_mn ? a_lbo : 16u, 1024u),
+                 smem_desc_sw128(b, b_mn ? b_lbo : 16u, 1024u), idesc, (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
+                      const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(sm);
+
+    __shared__ uint64_t bar_load, bar_ap, bar_c, bar_u, bar_os, bar_drain;
+    __shared__ uint32_t tmem_base_s;
+    __shared__ float s_beta[kC];
+    __shared__ float s_gammaC[kD];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3;           // TMEM lane quarter this warp may access
+    const int colhalf = warp >> 2;          // which 64 TMEM columns of a 128-wide result
+    const int bh = blockIdx.x;
+    const int b = bh / p.H, h = bh % p.H;
+    const int T = p.T;
+    const int nchunks = (T + kC - 1) / kC;
+
+    if (tid == 0) {
+        mbar_init(&bar_load, 1);
+        mbar_init(&bar_ap, 1);
+        mbar_init(&bar_c, 1);
+        mbar_init(&bar_u, 1);
+        mbar_init(&bar_os, 1);
+        mbar_init(&bar_drain, 1);
+        fence_mbar_init();
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_g);
+        prefetch_tensormap(&tm_v);
+    }
+    if (warp == 0) {
+        tmem_alloc(&tmem_base_s, TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tbase = tmem_base_s;
+    const uint32_t tlane = tbase + ((uint32_t)(32 * quarter) << 16);  // this warp's lane quarter
+
+    auto issue_loads = [&](int chunk) {
+        mbar_arrive_expect_tx(&bar_load, 4u * 16384u);
+        const int t0 = chunk * kC;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            tma_load_4d(sm + OFF_RAW_Q + x * 8192, &tm_q, &bar_load, 64 * x, h, t0, b);
+            tma_load_4d(sm + OFF_RAW_K + x * 8192, &tm_k, &bar_load, 64 * x, h, t0, b);
+            tma_load_4d(sm + OFF_RAW_G + x * 8192, &tm_g, &bar_load, 64 * x, h, t0, b);
+            tma_load_4d(sm + OFF_RAW_V + x * 8192, &tm_v, &bar_load, 64 * x, h, t0, b);
+        }
+    };
+    int pending_chunk = -1;  // chunk whose TMA loads are in flight (meaningful in thread 0)
+    if (tid == 0 && nchunks > 0) {
+        issue_loads(0);
+        pending_chunk = 0;
+    }
+
+    // ---- initial state: fp32 into TMEM (TM_S), bf16 copy into the MN-major S tile ----
+    {
+        const int i = 32 * quarter + lane;  // state row (dk index) = TMEM lane
+        for (int cb = 0; cb < 64; cb += 16) {
+            const int c0 = 64 * colhalf + cb;
+            float r[16];
+            if (p.S0) {
+                const float4* src = reinterpret_cast<const float4*>(p.S0 + ((size_t)bh * kD + i) * kD + c0);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float4 x = src[j];
+                    r[4 * j] = x.x; r[4 * j + 1] = x.y; r[4 * j + 2] = x.z; r[4 * j + 3] = x.w;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) r[j] = 0.f;
+            }
+            tmem_st16(tlane + TM_S + c0, r);
+#pragma unroll
+            for (int j = 0; j < 16; j += 8) {
+                uint4 pk;
+                pk.x = pack_bf16x2(r[j], r[j + 1]); pk.y = pack_bf16x2(r[j + 2], r[j + 3]);
+                pk.z = pack_bf16x2(r[j + 4], r[j + 5]); pk.w = pack_bf16x2(r[j + 6], r[j + 7]);
+                *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_offset(i, c0 + j, 16384)) = pk;
+            }
+        }
+        tmem_wait_st();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncthreads();
+
+    bool ok = true;
+    for (int chunk = 0; chunk < nchunks; ++chunk) {
+        const uint32_t par = chunk & 1;
+        const int t0 = chunk * kC;
+        const int nvalid = min(kC, T - t0);
+
+        if (tid < kC) {
+            const int t = t0 + tid;
+            s_beta[tid] = (t < T) ? __bfloat162float(p.beta[((size_t)b * T + t) * p.H + h]) : 0.f;
+        }
+        ok = mbar_wait(&bar_load, par, kTimeoutNs);
+        if (ok) pending_chunk = -1;
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok) break;
+
+        // ================= step 2: decay factors and the bf16 operand tiles =================
+        // thread = (channel i, half hf): tokens r = 32 hf + j, j = 0..31
+        const int ci = tid >> 1, hf = tid & 1;
+        uint32_t kb_pack[16];  // Kb values of this thread's 32 tokens (bf16x2), written after MMA1/2
+        {
+            const uint32_t ccol = (uint32_t)ci;
+            float G[32];
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                acc += bf16_at(sm + OFF_RAW_G, sw128_offset(32 * hf + j, ccol, 8192));
+                G[j] = acc;
+            }
+            const float other_total = __shfl_xor_sync(0xffffffffu, acc, 1);
+            if (hf == 1) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) G[j] += other_total;
+            }
+            const float my16 = G[16], my31 = G[31];
+            const float pr16 = __shfl_xor_sync(0xffffffffu, my16, 1);
+            const float pr31 = __shfl_xor_sync(0xffffffffu, my31, 1);
+            const float g16 = hf ? pr16 : my16, g31 = hf ? pr31 : my31;  // Gam_16, Gam_31
+            const float g48 = hf ? my16 : pr16, g63 = hf ? my31 : pr31;  // Gam_48, Gam_63
+            const float gm = hf ? g48 : g16;                              // mid reference of my block
+            const float cm = expf(gm);                 // e^{Gam_m}       (chunk-start reference)
+            const float ce = expf(g63 - gm);           // e^{Gam_63 - Gam_m}
+            const float c_off = hf ? expf(g48 - g31)   // block 1 rows: ref 48 -> ref 31
+                                   : expf(g31 - g16);  // block 0 cols: ref 16 -> ref 31
+            if (hf == 0) s_gammaC[ci] = expf(g63);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int r = 32 * hf + j;
+                const float x = G[j] - gm;
+                const float E = __expf(x), Ei = __expf(-x);
+                const uint32_t roff = sw128_offset(r, ccol, 8192);
+                const float qv = bf16_at(sm + OFF_RAW_Q, roff);
+                const float kv = bf16_at(sm + OFF_RAW_K, roff);
+                const float qE = qv * E, kE = kv * E, kEi = kv * Ei;
+                // MMA1 operands: rows [Qt0; Kt0; Qt1; Kt1] and [Kh0; Kh1] with mid references
+                put_bf16(sm + OFF_A1, sw128_offset(64 * hf + j, ccol, 16384), qE);
+                put_bf16(sm + OFF_A1, sw128_offset(64 * hf + 32 + j, ccol, 16384), kE);
+                put_bf16(sm + OFF_B1, sw128_offset(r, ccol, 8192), kEi);
+                if (hf) {  // MMA2 rows (block 1 against reference 31), stored as rows 64..127
+                    put_bf16(sm + OFF_A2, sw128_offset(j, ccol, 8192), qE * c_off);
+                    put_bf16(sm + OFF_A2, sw128_offset(32 + j, ccol, 8192), kE * c_off);
+                } else {   // MMA2 columns (block 0 against reference 31)
+                    put_bf16(sm + OFF_B2, sw128_offset(j, ccol, 4096), kEi * c_off);
+                }
+                // MMA3 operand [Kt; Qt] against the chunk start
+                put_bf16(sm + OFF_KQ, sw128_offset(r, ccol, 16384), kE * cm);
+                put_bf16(sm + OFF_KQ, sw128_offset(64 + r, ccol, 16384), qE * cm);
+                const float kbar = kEi * ce;
+                if (j & 1) kb_pack[j >> 1] |= (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(kbar)) << 16;
+                else kb_pack[j >> 1] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(kbar));
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        __syncthreads();
+
+        if (tid == 0) {
+            tc_fence_after_sync();
+            issue_mma(tbase + TM_AP, sb + OFF_A1, 16384, false, 0, sb + OFF_B1, 8192, false, 0, 8, ID_MMA1, false);
+            issue_mma(tbase + TM_AP + 64, sb + OFF_A2 - 8192, 8192, false, 0, sb + OFF_B2, 4096, false, 0, 8, ID_MMA2,
+                      false);
+            mma_commit(&bar_ap);
+            issue_mma(tbase + TM_C, sb + OFF_KQ, 16384, false, 0, sb + OFF_SB, 0, true, 16384, 8, ID_KxMN, false);
+            mma_commit(&bar_c);
+        }
+
+        // ================= step 3: P and A from TMEM, Kb tile =================
+        ok = mbar_wait(&bar_ap, par, kTimeoutNs);
+        tc_fence_after_sync();
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok) break;
+        {
+            // Kb (MN-major A of MMA6: row = token j, column = channel i)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const uint16_t bits = (uint16_t)((kb_pack[j >> 1] >> ((j & 1) * 16)) & 0xFFFFu);
+                *reinterpret_cast<uint16_t*>(sm + OFF_KBAR + sw128_offset(32 * hf + j, (uint32_t)ci, 8192)) = bits;
+            }
+        }
+        if (warp < 4) {
+            // lane L of TM_AP: L < 32: Qt0 row r = L; L < 64: Kt0 row r = L - 32;
+            //                  L < 96: Qt1 row r = L - 32; else Kt1 row r = L - 64.
+            const int L = 32 * warp + lane;
+            const bool is_q = (L < 32) || (L >= 64 && L < 96);
+            const int r = (L < 64) ? (L & 31) : 32 + (L & 31);
+            float row[64];
+            if (r < 32) {
+#pragma unroll
+                for (int cb = 0; cb < 32; cb += 16) tmem_ld16(tlane + TM_AP + cb, row + cb);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 32; j < 64; ++j) row[j] = 0.f;
+            } else {
+                float dg[32];
+                // MMA2 columns 0..31 hold the off-diagonal block (cols j = 0..31)
+#pragma unroll
+                for (int cb = 0; cb < 32; cb += 16) tmem_ld16(tlane + TM_AP + 64 + cb, row + cb);
+                // MMA1 columns 32..63 hold the diagonal block of block 1 (cols j = 32..63)
+#pragma unroll
+                for (int cb = 0; cb < 32; cb += 16) tmem_ld16(tlane + TM_AP + 32 + cb, dg + cb);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) row[32 + j] = dg[j];
+            }
+            if (is_q) {
+                // P row r: lower triangle including the diagonal, bf16, K-major rows 64.. of the P tile
+#pragma unroll
+                for (int j = 0; j < 64; j += 8) {
+                    uint4 pk;
+                    float v8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v8[e] = (j + e <= r) ? row[j + e] : 0.f;
+                    pk.x = pack_bf16x2(v8[0], v8[1]); pk.y = pack_bf16x2(v8[2], v8[3]);
+                    pk.z = pack_bf16x2(v8[4], v8[5]); pk.w = pack_bf16x2(v8[6], v8[7]);
+                    *reinterpret_cast<uint4*>(sm + OFF_PV + 8192 + sw128_offset(r, j, 8192)) = pk;
+                }
+            } else {
+                // A row r: strictly lower, scaled by beta_r, fp32 row-major for the solve
+                const float br = s_beta[r];
+                float* arow = reinterpret_cast<float*>(sm + OFF_AF) + r * 64;
+#pragma unroll
+                for (int j = 0; j < 64; j += 4) {
+                    float4 w;
+                    w.x = (j + 0 < r) ? br * row[j + 0] : 0.f;
+                    w.y = (j + 1 < r) ? br * row[j + 1] : 0.f;
+                    w.z = (j + 2 < r) ? br * row[j + 2] : 0.f;
+                    w.w = (j + 3 < r) ? br * row[j + 3] : 0.f;
+                    *reinterpret_cast<float4*>(arow + j) = w;
+                }
+            }
+        }
+        __syncthreads();
+
+        // ================= step 4: X = (I + A)^{-1} (fp32, 16x16 blocks), T = X Diag(beta) ==========
+        {
+            const float* Am = reinterpret_cast<const float*>(sm + OFF_AF);
+            float* X = reinterpret_cast<float*>(sm + OFF_X);
+            float* W = reinterpret_cast<float*>(sm + OFF_W);
+            // diagonal blocks by forward substitution, one thread per (block, column)
+            if (tid < 64) {
+                const int bb = tid >> 4, c = tid & 15, o0 = 16 * bb;
+                float x[16];
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) {
+                    float s = (rr == c) ? 1.f : 0.f;
+#pragma unroll
+                    for (int l = 0; l < rr; ++l) s -= Am[(o0 + rr) * 64 + o0 + l] * x[l];
+                    x[rr] = (rr < c) ? 0.f : s;
+                }
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) X[(o0 + rr) * 64 + o0 + c] = x[rr];
+            } else if (tid < 128) {
+                // zero the strictly upper blocks of X
+                const int t = tid - 64;
+                for (int e = t; e < 64 * 64; e += 64) {
+                    const int rr = e >> 6, cc = e & 63;
+                    if ((cc >> 4) > (rr >> 4)) X[e] = 0.f;
+                }
+            }
+            __syncthreads();
+            // off-diagonal blocks, by distance d = R - J: X_RJ = -X_RR sum_{L=J}^{R-1} A_RL X_LJ
+            const int er = tid >> 4, ec = tid & 15;
+#pragma unroll 1
+            for (int d = 1; d < 4; ++d) {
+                const int nblk = 4 - d;
+                for (int q = 0; q < nblk; ++q) {
+                    const int R = q + d, J = q;
+                    float s = 0.f;
+                    for (int L = J; L < R; ++L)
+#pragma unroll
+                        for (int l = 0; l < 16; ++l)
+                            s += Am[(16 * R + er) * 64 + 16 * L + l] * X[(16 * L + l) * 64 + 16 * J + ec];
+                    W[q * 256 + er * 16 + ec] = s;
+                }
+                __syncthreads();
+                for (int q = 0; q < nblk; ++q) {
+                    const int R = q + d, J = q;
+                    float s = 0.f;
+#pragma unroll
+                    for (int l = 0; l < 16; ++l) s -= X[(16 * R + er) * 64 + 16 * R + l] * W[q * 256 + l * 16 + ec];
+                    X[(16 * R + er) * 64 + 16 * J + ec] = s;
+                }
+                __syncthreads();
+            }
+            // T = X Diag(beta) -> bf16 K-major tile rows 0..63 (K = 64 tokens)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int idx = tid + kThreads * e;  // 512 chunks of 8
+                const int r = idx >> 3, j = (idx & 7) * 8;
+                const float* xr = X + r * 64 + j;
+                uint4 pk;
+                pk.x = pack_bf16x2(xr[0] * s_beta[j + 0], xr[1] * s_beta[j + 1]);
+                pk.y = pack_bf16x2(xr[2] * s_beta[j + 2], xr[3] * s_beta[j + 3]);
+                pk.z = pack_bf16x2(xr[4] * s_beta[j + 4], xr[5] * s_beta[j + 5]);
+                pk.w = pack_bf16x2(xr[6] * s_beta[j + 6], xr[7] * s_beta[j + 7]);
+                *reinterpret_cast<uint4*>(sm + OFF_T + sw128_offset(r, j, 8192)) = pk;
+            }
+        }
+
+        // ================= step 5: Y = V - Kt S  (TMEM lanes 0..63 of TM_C) =================
+        ok = mbar_wait(&bar_c, par, kTimeoutNs);
+        tc_fence_after_sync();
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok) break;
+        if (quarter < 2) {
+            const int r = 32 * quarter + lane;
+#pragma unroll
+            for (int cb = 0; cb < 64; cb += 16) {
+                const int c0 = 64 * colhalf + cb;
+                float ks[16];
+                tmem_ld16(tlane + TM_C + c0, ks);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; j += 8) {
+                    const uint32_t off = sw128_offset(r, c0 + j, 8192);
+                    const uint4 vv = *reinterpret_cast<const uint4*>(sm + OFF_RAW_V + off);
+                    const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vv);
+                    uint4 pk;
+                    float2 f;
+                    f = __bfloat1622float2(v2[0]); pk.x = pack_bf16x2(f.x - ks[j + 0], f.y - ks[j + 1]);
+                    f = __bfloat1622float2(v2[1]); pk.y = pack_bf16x2(f.x - ks[j + 2], f.y - ks[j + 3]);
+                    f = __bfloat1622float2(v2[2]); pk.z = pack_bf16x2(f.x - ks[j + 4], f.y - ks[j + 5]);
+                    f = __bfloat1622float2(v2[3]); pk.w = pack_bf16x2(f.x - ks[j + 6], f.y - ks[j + 7]);
+                    *reinterpret_cast<uint4*>(sm + OFF_YU + off) = pk;
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after_sync();
+            // raw tiles are all consumed: prefetch the next chunk
+            if (chunk + 1 < nchunks) {
+                issue_loads(chunk + 1);
+                pending_chunk = chunk + 1;
+            }
+            issue_mma(tbase + TM_U, sb + OFF_T, 0, false, 0, sb + OFF_YU, 0, true, 8192, 4, ID_KxMN, false);
+            mma_commit(&bar_u);
+        }
+
+        // ================= step 7: decay the fp32 state in TMEM; U -> bf16 tile =================
+        {
+#pragma unroll
+            for (int cb = 0; cb < 64; cb += 16) {
+                const int c0 = 64 * colhalf + cb;
+                float sv[16];
+                tmem_ld16(tlane + TM_S + c0, sv);
+                tmem_wait_ld();
+                const float gc = s_gammaC[32 * quarter + lane];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) sv[j] *= gc;
+                tmem_st16(tlane + TM_S + c0, sv);
+            }
+            tmem_wait_st();
+        }
+        ok = mbar_wait(&bar_u, par, kTimeoutNs);
+        tc_fence_after_sync();
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok) break;
+        if (quarter < 2) {
+            const int r = 32 * quarter + lane;
+#pragma unroll
+            for (int cb = 0; cb < 64; cb += 16) {
+                const int c0 = 64 * colhalf + cb;
+                float u[16];
+                tmem_ld16(tlane + TM_U + c0, u);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; j += 8) {
+                    uint4 pk;
+                    pk.x = pack_bf16x2(u[j], u[j + 1]); pk.y = pack_bf16x2(u[j + 2], u[j + 3]);
+                    pk.z = pack_bf16x2(u[j + 4], u[j + 5]); pk.w = pack_bf16x2(u[j + 6], u[j + 7]);
+                    *reinterpret_cast<uint4*>(sm + OFF_YU + sw128_offset(r, c0 + j, 8192)) = pk;
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after_sync();
+            // O = Qt S + P U (onto lanes 64..127 of TM_C); S <- Diag(gamma_C) S + Kb^T U
+            issue_mma(tbase + TM_C, sb + OFF_PV, 0, false, 0, sb + OFF_YU, 0, true, 8192, 4, ID_KxMN, true);
+            issue_mma(tbase + TM_S, sb + OFF_KBAR, 0, true, 8192, sb + OFF_YU, 0, true, 8192, 4, ID_MNxMN, true);
+            mma_commit(&bar_os);
+        }
+
+        // ================= step 9: O -> global; S -> bf16 tile for the next chunk =================
+        ok = mbar_wait(&bar_os, par, kTimeoutNs);
+        tc_fence_after_sync();
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok) break;
+        if (quarter >= 2) {
+            const int r = 32 * (quarter - 2) + lane;
+            // tcgen05.ld is warp-collective: every lane loads, only valid tokens are stored
+            const bool valid = r < nvalid;
+            __nv_bfloat16* orow = p.o + (((size_t)b * T + t0 + (valid ? r : 0)) * p.H + h) * kD;
+#pragma unroll
+            for (int cb = 0; cb < 64; cb += 16) {
+                const int c0 = 64 * colhalf + cb;
+                float ov[16];
+                tmem_ld16(tlane + TM_C + c0, ov);
+                tmem_wait_ld();
+                if (valid) {
+                    uint4 pk0, pk1;
+                    pk0.x = pack_bf16x2(ov[0], ov[1]); pk0.y = pack_bf16x2(ov[2], ov[3]);
+                    pk0.z = pack_bf16x2(ov[4], ov[5]); pk0.w = pack_bf16x2(ov[6], ov[7]);
+                    pk1.x = pack_bf16x2(ov[8], ov[9]); pk1.y = pack_bf16x2(ov[10], ov[11]);
+                    pk1.z = pack_bf16x2(ov[12], ov[13]); pk1.w = pack_bf16x2(ov[14], ov[15]);
+                    *reinterpret_cast<uint4*>(orow + c0) = pk0;
+                    *reinterpret_cast<uint4*>(orow + c0 + 8) = pk1;
+                }
+            }
+        }
+        {
+            const int i = 32 * quarter + lane;
+#pragma unroll
+            for (int cb = 0; cb < 64; cb += 16) {
+                const int c0 = 64 * colhalf + cb;
+                float sv[16];
+                tmem_ld16(tlane + TM_S + c0, sv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; j += 8) {
+                    uint4 pk;
+                    pk.x = pack_bf16x2(sv[j], sv[j + 1]); pk.y = pack_bf16x2(sv[j + 2], sv[j + 3]);
+                    pk.z = pack_bf16x2(sv[j + 4], sv[j + 5]); pk.w = pack_bf16x2(sv[j + 6], sv[j + 7]);
+                    *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_offset(i, c0 + j, 16384)) = pk;
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        __syncthreads();
+    }
+
+    if (!ok && tid == 0) report_status(p.status, KDA_ERR_TIMEOUT);
+    // ---- drain: no tensor-core work or TMA may be in flight when the CTA exits ----
+    if (tid == 0) {
+        mma_commit(&bar_drain);
+        if (!mbar_wait(&bar_drain, 0, kTimeoutNs)) report_status(p.status, KDA_ERR_TIMEOUT);
+        if (pending_chunk >= 0) {
+            // a prefetch may still be landing: wait for it (bounded) before the smem is released
+            (void)mbar_wait(&bar_load, (uint32_t)(pending_chunk & 1), kTimeoutNs);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (ok && p.ST) {
+        const int i = 32 * quarter + lane;
+        float* dst = p.ST + ((size_t)bh * kD + i) * kD;
+#pragma unroll
+        for (int cb = 0; cb < 64; cb += 16) {
+            const int c0 = 64 * colhalf + cb;
+            float sv[16];
+            tmem_ld16(tlane + TM_S + c0, sv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; j += 4)
+                *reinterpret_cast<float4*>(dst + c0 + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, TM_COLS);
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// [B, T, H, 128] bf16 viewed as a 4-D tensor (d, H, T, B); box = 64 channels x 1 head x 64 tokens.
+bool make_map(CUtensorMap* m, const void* ptr, int B, int T, int H) {
+    auto enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)T * H * kD * 2};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)kC, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool prefill_tc_supports(const PrefillArgs& a) {
+    return a.dtype == KDA_DTYPE_BF16 && a.dk == kD && a.dv == kD;
+}
+
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
+    static std::mutex mu;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (dev < 64 && !attr_set[dev]) {
+            e = cudaFuncSetAttribute(kda_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
+            if (e != cudaSuccess) return e;
+            attr_set[dev] = true;
+        }
+    }
+    CUtensorMap mq, mk, mg, mv;
+    if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
+        !make_map(&mg, a.g, a.B, a.T, a.H) || !make_map(&mv, a.v, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
+    TcParams prm{static_cast<const __nv_bfloat16*>(a.beta), a.S0, static_cast<__nv_bfloat16*>(a.o), a.ST,
+                 a.status, a.B, a.T, a.H};
+    kda_prefill_tc_kernel<<<(unsigned)((size_t)a.B * a.H), kThreads, SMEM_DYN, s>>>(mq, mk, mg, mv, prm);
+    return cudaGetLastError();
+}
+
 }  // namespace kda
