@@ -66,8 +66,16 @@ constexpr uint32_t OFF_KQ = OFF_AP + 73728;         // [Kt; Qt], K-major, 128 ro
 constexpr uint32_t OFF_SB = OFF_KQ + 32768;         // S in bf16, MN-major B (K = dk), 2 atoms x 16 KB
 constexpr uint32_t OFF_YU = OFF_SB + 32768;         // Y then U, MN-major B (K = 64), 2 atoms x 8 KB
 constexpr uint32_t SMEM_BYTES = OFF_YU + 16384;     // 221184
-constexpr uint32_t OFF_X = OFF_RAW_Q;               // solve: X = (I+A)^-1, fp32 64x64 (raw q is dead)
-constexpr uint32_t OFF_W = OFF_RAW_K;               // solve scratch, fp32 3 x 16x16
+constexpr uint32_t OFF_L = OFF_AP + 8192;           // chunk start: lower-triangular ones (8 KB)
+constexpr uint32_t OFF_CONST = OFF_YU;              // step 2: reference rows of Gam + per-channel constants
+constexpr int kLd = 68;                             // padded row stride (floats) of the solve matrices
+constexpr uint32_t OFF_X = OFF_RAW_Q;               // solve: X = (I+A)^-1 fp32 (raw q/k/g are dead)
+constexpr uint32_t OFF_XT = OFF_X + 64 * kLd * 4;   //   X transposed
+constexpr int kLdS = 20;
+constexpr uint32_t OFF_WS = OFF_XT + 64 * kLd * 4;  //   per-warp W^T scratch (8 warps x 8 x kLdS)
+static_assert(OFF_WS + 8 * 8 * kLdS * 4 <= OFF_RAW_V, "solve scratch overlaps raw v");
+static_assert(OFF_AF + 64 * kLd * 4 <= OFF_KQ, "A overlaps the KQ tile");
+constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t SMEM_DYN = SMEM_BYTES + 1024;    // + alignment slack
 
 // ---- TMEM columns (fp32 accumulators, 128 lanes) ----
@@ -81,6 +89,7 @@ constexpr uint32_t ID_MMA1 = idesc_bf16_f32(128, 64, false, false);
 constexpr uint32_t ID_MMA2 = idesc_bf16_f32(128, 32, false, false);
 constexpr uint32_t ID_KxMN = idesc_bf16_f32(128, 128, false, true);
 constexpr uint32_t ID_MNxMN = idesc_bf16_f32(128, 128, true, true);
+constexpr uint32_t ID_G = idesc_bf16_f32(128, 64, false, true);
 
 struct TcParams {
     const __nv_bfloat16* beta;
@@ -95,26 +104,58 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&p);
 }
-__device__ __forceinline__ float bf16_at(const uint8_t* base, uint32_t off) {
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
-}
-__device__ __forceinline__ void put_bf16(uint8_t* base, uint32_t off, float x) {
-    *reinterpret_cast<__nv_bfloat16*>(base + off) = __float2bfloat16_rn(x);
+
+// Byte offset of K step kk (16 elements) inside an operand tile: K-major tiles advance 32 B
+// inside a 128-byte swizzle row and jump to the next 64-column atom every 4 steps; MN-major
+// tiles advance 16 rows (2048 B).
+template <bool MN, uint32_t ATOM>
+__device__ __forceinline__ constexpr uint32_t kstep_off(int kk) {
+    return MN ? (uint32_t)kk * 2048u : (uint32_t)(kk >> 2) * ATOM + (uint32_t)(kk & 3) * 32u;
 }
 
-// Issue one K-major-A / any-B product of K = 16*ksteps.  a_atom / b_atom: byte distance
-// between 64-column K atoms of a K-major operand; b_mn: B is MN-major (then b_lbo is the
-// distance between its 64-wide N atoms and each K step advances 16 rows = 2048 B).
-__device__ __forceinline__ void issue_mma(uint32_t d_tmem, uint32_t a_base, uint32_t a_atom, bool a_mn,
-                                          uint32_t a_lbo, uint32_t b_base, uint32_t b_atom, bool b_mn,
-                                          uint32_t b_lbo, int ksteps, uint32_t idesc, bool accumulate) {
-#pragma unroll 1
-    for (int kk = 0; kk < ksteps; ++kk) {
-        const uint32_t a = a_mn ? a_base + kk * 2048u : a_base + (kk >> 2) * a_atom + (kk & 3) * 32u;
-        const uint32_t b = b_mn ? b_base + kk * 2048u : b_base + (kk >> 2) * b_atom + (kk & 3) * 32u;
-        mma_bf16(d_tmem, smem_desc_sw128(a, a_mn ? a_lbo : 16u, 1024u),
-                 smem_desc_sw128(b, b_mn ? b_lbo : 16u, 1024u), idesc, (accumulate || kk > 0) ? 1u : 0u);
-    }
+// Issue D (+)= A * B over K = 16 * KSTEPS from one thread.  Descriptors are built once and
+// advanced by constant offsets (the start-address field is the low 14 bits, in 16-byte units).
+template <int KSTEPS, bool A_MN, uint32_t A_ATOM, bool B_MN, uint32_t B_ATOM>
+__device__ __forceinline__ void issue_mma(uint32_t d_tmem, uint32_t a_base, uint32_t b_base, uint32_t idesc,
+                                          bool accumulate) {
+    const uint64_t ad = smem_desc_sw128(a_base, A_MN ? A_ATOM : 16u, 1024u);
+    const uint64_t bd = smem_desc_sw128(b_base, B_MN ? B_ATOM : 16u, 1024u);
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk)
+        mma_bf16(d_tmem, ad + (kstep_off<A_MN, A_ATOM>(kk) >> 4), bd + (kstep_off<B_MN, B_ATOM>(kk) >> 4), idesc,
+                 (kk > 0 || accumulate) ? 1u : 0u);
+}
+
+// Warp-level bf16 tensor-core tile D(16x8) += A(16x16, row-major) * B(16x8, column-major), fp32
+// accumulate.  Fragment ownership (lane = 4*g + t): A {(g,2t..2t+1), (g+8,2t..), (g,2t+8..), (g+8,2t+8..)},
+// B {(2t..2t+1, g), (2t+8.., g)}, D {(g,2t), (g,2t+1), (g+8,2t), (g+8,2t+1)}.
+__device__ __forceinline__ void mma_16816(float d[4], const uint32_t a[4], const uint32_t b[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// A fragment from a row-major fp32 16x16 block (row stride ld floats), rounded to bf16.
+__device__ __forceinline__ void load_a_frag(const float* blk, int ld, int g, int t, uint32_t a[4]) {
+    const float2 v0 = *reinterpret_cast<const float2*>(blk + g * ld + 2 * t);
+    const float2 v1 = *reinterpret_cast<const float2*>(blk + (g + 8) * ld + 2 * t);
+    const float2 v2 = *reinterpret_cast<const float2*>(blk + g * ld + 2 * t + 8);
+    const float2 v3 = *reinterpret_cast<const float2*>(blk + (g + 8) * ld + 2 * t + 8);
+    a[0] = pack_bf16x2(v0.x, v0.y); a[1] = pack_bf16x2(v1.x, v1.y);
+    a[2] = pack_bf16x2(v2.x, v2.y); a[3] = pack_bf16x2(v3.x, v3.y);
+}
+// B fragment of a 16x8 (K x N) block stored transposed (row n holds the 16 K values), rounded to bf16.
+__device__ __forceinline__ void load_b_frag(const float* blkT, int ld, int g, int t, uint32_t b[2]) {
+    const float2 v0 = *reinterpret_cast<const float2*>(blkT + g * ld + 2 * t);
+    const float2 v1 = *reinterpret_cast<const float2*>(blkT + g * ld + 2 * t + 8);
+    b[0] = pack_bf16x2(v0.x, v0.y); b[1] = pack_bf16x2(v1.x, v1.y);
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -122,10 +163,13 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                       const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
                       const TcParams p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // Align to 1024 B (the swizzle atoms need it) by offsetting the shared array itself, so the
+    // compiler keeps every access in the shared state space.
+    const uint32_t raw_base = smem_u32(smem_raw);
+    uint8_t* sm = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);
     const uint32_t sb = smem_u32(sm);
 
-    __shared__ uint64_t bar_load, bar_ap, bar_c, bar_u, bar_os, bar_drain;
+    __shared__ uint64_t bar_load, bar_g, bar_ap, bar_c, bar_u, bar_os, bar_drain;
     __shared__ uint32_t tmem_base_s;
     __shared__ float s_beta[kC];
     __shared__ float s_gammaC[kD];
@@ -140,6 +184,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
     if (tid == 0) {
         mbar_init(&bar_load, 1);
+        mbar_init(&bar_g, 1);
         mbar_init(&bar_ap, 1);
         mbar_init(&bar_c, 1);
         mbar_init(&bar_u, 1);
@@ -220,65 +265,135 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const int t = t0 + tid;
             s_beta[tid] = (t < T) ? __bfloat162float(p.beta[((size_t)b * T + t) * p.H + h]) : 0.f;
         }
+        // Lower-triangular ones L[r][j] = (j <= r), bf16, K-major, 64 rows: the in-chunk cumulative
+        // sum of g as a tensor-core product (Gam = L g).  Rewritten every chunk because its home in
+        // the operand region is reused later in the chunk.
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int idx = tid + kThreads * e;  // 512 chunks of 8 elements
+            const int r = idx >> 3, j0 = (idx & 7) * 8;
+            uint4 pk;
+            uint32_t w[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const uint32_t lo = (j0 + 2 * m <= r) ? 0x3F80u : 0u;
+                const uint32_t hi = (j0 + 2 * m + 1 <= r) ? 0x3F80u : 0u;
+                w[m] = lo | (hi << 16);
+            }
+            pk.x = w[0]; pk.y = w[1]; pk.z = w[2]; pk.w = w[3];
+            *reinterpret_cast<uint4*>(sm + OFF_L + sw128_offset(r, j0, 8192)) = pk;
+        }
+        fence_proxy_async_smem();
         ok = mbar_wait(&bar_load, par, kTimeoutNs);
         if (ok) pending_chunk = -1;
         ok = __syncthreads_and(ok) != 0;
         if (!ok) break;
+        if (tid == 0) {
+            tc_fence_after_sync();
+            // Gam for channels 0..63 into lanes 0..63 (rows 64..127 of A read other smem),
+            // channels 64..127 into lanes 64..127 (rows 0..63 of A read other smem)
+            issue_mma<4, false, 0, true, 8192>(tbase + TM_U, sb + OFF_L, sb + OFF_RAW_G, ID_G, false);
+            issue_mma<4, false, 0, true, 8192>(tbase + TM_U + 64, sb + OFF_L - 8192, sb + OFF_RAW_G + 8192, ID_G, false);
+            mma_commit(&bar_g);
+        }
 
         // ================= step 2: decay factors and the bf16 operand tiles =================
-        // thread = (channel i, half hf): tokens r = 32 hf + j, j = 0..31
-        const int ci = tid >> 1, hf = tid & 1;
-        uint32_t kb_pack[16];  // Kb values of this thread's 32 tokens (bf16x2), written after MMA1/2
+        // thread = one token row r and 32 channels c0..c0+31 (its TMEM lane holds Gam[r][c0..])
+        const int tr = 32 * (quarter & 1) + lane;            // token
+        const int hf = quarter & 1;                          // 32-token block of the token
+        const int jr = lane;                                 // row inside the block
+        const int c0 = 64 * (quarter >> 1) + 32 * colhalf;   // first channel
+        float* refs = reinterpret_cast<float*>(sm + OFF_CONST);          // [4][128] Gam rows 16,31,48,63
+        float* cst = refs + 4 * kD;                                       // per-channel constants
+        // cst layout: [hf][k][128] with k = 0: Gam_m*log2e, 1: e^{Gam_m}, 2: e^{Gam_63-Gam_m}, 3: c_off
+        uint32_t kb[16];  // Kb of this token row, bf16x2, stored once MMA1/2 have finished reading B1
         {
-            const uint32_t ccol = (uint32_t)ci;
+            ok = mbar_wait(&bar_g, par, kTimeoutNs);
+            tc_fence_after_sync();
             float G[32];
-            float acc = 0.f;
+            tmem_ld16(tlane + TM_U + c0, G);          // lanes 64.. hold channels 64.. (second MMA)
+            tmem_ld16(tlane + TM_U + c0 + 16, G + 16);
+            tmem_wait_ld();
+            const int refk = (lane == 16) ? 0 : (lane == 31) ? 1 : -1;
+            if (refk >= 0) {
+                float* dst = refs + (2 * hf + refk) * kD + c0;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                acc += bf16_at(sm + OFF_RAW_G, sw128_offset(32 * hf + j, ccol, 8192));
-                G[j] = acc;
+                for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(G[e], G[e + 1], G[e + 2], G[e + 3]);
             }
-            const float other_total = __shfl_xor_sync(0xffffffffu, acc, 1);
-            if (hf == 1) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) G[j] += other_total;
+            ok = __syncthreads_and(ok) != 0;
+            if (!ok) break;
+            if (tid < kD) {
+                const float g16 = refs[tid], g31 = refs[kD + tid], g48 = refs[2 * kD + tid], g63 = refs[3 * kD + tid];
+                cst[0 * kD + tid] = g16 * kLog2e;
+                cst[1 * kD + tid] = expf(g16);
+                cst[2 * kD + tid] = expf(g63 - g16);
+                cst[3 * kD + tid] = expf(g31 - g16);
+                cst[4 * kD + tid] = g48 * kLog2e;
+                cst[5 * kD + tid] = expf(g48);
+                cst[6 * kD + tid] = expf(g63 - g48);
+                cst[7 * kD + tid] = expf(g48 - g31);
+                s_gammaC[tid] = expf(g63);
             }
-            const float my16 = G[16], my31 = G[31];
-            const float pr16 = __shfl_xor_sync(0xffffffffu, my16, 1);
-            const float pr31 = __shfl_xor_sync(0xffffffffu, my31, 1);
-            const float g16 = hf ? pr16 : my16, g31 = hf ? pr31 : my31;  // Gam_16, Gam_31
-            const float g48 = hf ? my16 : pr16, g63 = hf ? my31 : pr31;  // Gam_48, Gam_63
-            const float gm = hf ? g48 : g16;                              // mid reference of my block
-            const float cm = expf(gm);                 // e^{Gam_m}       (chunk-start reference)
-            const float ce = expf(g63 - gm);           // e^{Gam_63 - Gam_m}
-            const float c_off = hf ? expf(g48 - g31)   // block 1 rows: ref 48 -> ref 31
-                                   : expf(g31 - g16);  // block 0 cols: ref 16 -> ref 31
-            if (hf == 0) s_gammaC[ci] = expf(g63);
+            __syncthreads();
+            const float* ch = cst + 4 * kD * hf;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int r = 32 * hf + j;
-                const float x = G[j] - gm;
-                const float E = __expf(x), Ei = __expf(-x);
-                const uint32_t roff = sw128_offset(r, ccol, 8192);
-                const float qv = bf16_at(sm + OFF_RAW_Q, roff);
-                const float kv = bf16_at(sm + OFF_RAW_K, roff);
-                const float qE = qv * E, kE = kv * E, kEi = kv * Ei;
-                // MMA1 operands: rows [Qt0; Kt0; Qt1; Kt1] and [Kh0; Kh1] with mid references
-                put_bf16(sm + OFF_A1, sw128_offset(64 * hf + j, ccol, 16384), qE);
-                put_bf16(sm + OFF_A1, sw128_offset(64 * hf + 32 + j, ccol, 16384), kE);
-                put_bf16(sm + OFF_B1, sw128_offset(r, ccol, 8192), kEi);
-                if (hf) {  // MMA2 rows (block 1 against reference 31), stored as rows 64..127
-                    put_bf16(sm + OFF_A2, sw128_offset(j, ccol, 8192), qE * c_off);
-                    put_bf16(sm + OFF_A2, sw128_offset(32 + j, ccol, 8192), kE * c_off);
-                } else {   // MMA2 columns (block 0 against reference 31)
-                    put_bf16(sm + OFF_B2, sw128_offset(j, ccol, 4096), kEi * c_off);
+            for (int g8 = 0; g8 < 4; ++g8) {
+                const int cc = c0 + 8 * g8;
+                const uint32_t roff = sw128_offset(tr, cc, 8192);
+                const uint4 qraw = *reinterpret_cast<const uint4*>(sm + OFF_RAW_Q + roff);
+                const uint4 kraw = *reinterpret_cast<const uint4*>(sm + OFF_RAW_K + roff);
+                float gmL[8], cm[8], ce[8], co[8];
+                *reinterpret_cast<float4*>(gmL) = *reinterpret_cast<const float4*>(ch + 0 * kD + cc);
+                *reinterpret_cast<float4*>(gmL + 4) = *reinterpret_cast<const float4*>(ch + 0 * kD + cc + 4);
+                *reinterpret_cast<float4*>(cm) = *reinterpret_cast<const float4*>(ch + 1 * kD + cc);
+                *reinterpret_cast<float4*>(cm + 4) = *reinterpret_cast<const float4*>(ch + 1 * kD + cc + 4);
+                *reinterpret_cast<float4*>(ce) = *reinterpret_cast<const float4*>(ch + 2 * kD + cc);
+                *reinterpret_cast<float4*>(ce + 4) = *reinterpret_cast<const float4*>(ch + 2 * kD + cc + 4);
+                *reinterpret_cast<float4*>(co) = *reinterpret_cast<const float4*>(ch + 3 * kD + cc);
+                *reinterpret_cast<float4*>(co + 4) = *reinterpret_cast<const float4*>(ch + 3 * kD + cc + 4);
+                const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qraw);
+                const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kraw);
+                uint32_t a1q[4], a1k[4], b1[4], kqk[4], kqq[4], x1[4], x2[4];
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const float2 qf = __bfloat1622float2(q2[m]);
+                    const float2 kf = __bfloat1622float2(k2[m]);
+                    float E[2], Ei[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const float xl = fmaf(G[8 * g8 + 2 * m + u], kLog2e, -gmL[2 * m + u]);
+                        E[u] = ex2_approx(xl);
+                        Ei[u] = ex2_approx(-xl);
+                    }
+                    const float qE0 = qf.x * E[0], qE1 = qf.y * E[1];
+                    const float kE0 = kf.x * E[0], kE1 = kf.y * E[1];
+                    const float kI0 = kf.x * Ei[0], kI1 = kf.y * Ei[1];
+                    a1q[m] = pack_bf16x2(qE0, qE1);
+                    a1k[m] = pack_bf16x2(kE0, kE1);
+                    b1[m] = pack_bf16x2(kI0, kI1);
+                    kqk[m] = pack_bf16x2(kE0 * cm[2 * m], kE1 * cm[2 * m + 1]);
+                    kqq[m] = pack_bf16x2(qE0 * cm[2 * m], qE1 * cm[2 * m + 1]);
+                    kb[4 * g8 + m] = pack_bf16x2(kI0 * ce[2 * m], kI1 * ce[2 * m + 1]);
+                    if (hf) {
+                        x1[m] = pack_bf16x2(qE0 * co[2 * m], qE1 * co[2 * m + 1]);
+                        x2[m] = pack_bf16x2(kE0 * co[2 * m], kE1 * co[2 * m + 1]);
+                    } else {
+                        x1[m] = pack_bf16x2(kI0 * co[2 * m], kI1 * co[2 * m + 1]);
+                    }
                 }
+                // MMA1 operands: rows [Qt0; Kt0; Qt1; Kt1] and [Kh0; Kh1] against the block middles
+                *reinterpret_cast<uint4*>(sm + OFF_A1 + sw128_offset(64 * hf + jr, cc, 16384)) = make_uint4(a1q[0], a1q[1], a1q[2], a1q[3]);
+                *reinterpret_cast<uint4*>(sm + OFF_A1 + sw128_offset(64 * hf + 32 + jr, cc, 16384)) = make_uint4(a1k[0], a1k[1], a1k[2], a1k[3]);
+                *reinterpret_cast<uint4*>(sm + OFF_B1 + sw128_offset(tr, cc, 8192)) = make_uint4(b1[0], b1[1], b1[2], b1[3]);
                 // MMA3 operand [Kt; Qt] against the chunk start
-                put_bf16(sm + OFF_KQ, sw128_offset(r, ccol, 16384), kE * cm);
-                put_bf16(sm + OFF_KQ, sw128_offset(64 + r, ccol, 16384), qE * cm);
-                const float kbar = kEi * ce;
-                if (j & 1) kb_pack[j >> 1] |= (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(kbar)) << 16;
-                else kb_pack[j >> 1] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(kbar));
+                *reinterpret_cast<uint4*>(sm + OFF_KQ + sw128_offset(tr, cc, 16384)) = make_uint4(kqk[0], kqk[1], kqk[2], kqk[3]);
+                *reinterpret_cast<uint4*>(sm + OFF_KQ + sw128_offset(64 + tr, cc, 16384)) = make_uint4(kqq[0], kqq[1], kqq[2], kqq[3]);
+                if (hf) {  // MMA2 rows: block 1 against token 31, stored as rows 64..127 of a virtual tile
+                    *reinterpret_cast<uint4*>(sm + OFF_A2 + sw128_offset(jr, cc, 8192)) = make_uint4(x1[0], x1[1], x1[2], x1[3]);
+                    *reinterpret_cast<uint4*>(sm + OFF_A2 + sw128_offset(32 + jr, cc, 8192)) = make_uint4(x2[0], x2[1], x2[2], x2[3]);
+                } else {   // MMA2 columns: block 0 against token 31
+                    *reinterpret_cast<uint4*>(sm + OFF_B2 + sw128_offset(jr, cc, 4096)) = make_uint4(x1[0], x1[1], x1[2], x1[3]);
+                }
             }
         }
         fence_proxy_async_smem();
@@ -287,143 +402,157 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
         if (tid == 0) {
             tc_fence_after_sync();
-            issue_mma(tbase + TM_AP, sb + OFF_A1, 16384, false, 0, sb + OFF_B1, 8192, false, 0, 8, ID_MMA1, false);
-            issue_mma(tbase + TM_AP + 64, sb + OFF_A2 - 8192, 8192, false, 0, sb + OFF_B2, 4096, false, 0, 8, ID_MMA2,
-                      false);
+            issue_mma<8, false, 16384, false, 8192>(tbase + TM_AP, sb + OFF_A1, sb + OFF_B1, ID_MMA1, false);
+            issue_mma<8, false, 8192, false, 4096>(tbase + TM_AP + 64, sb + OFF_A2 - 8192, sb + OFF_B2, ID_MMA2, false);
             mma_commit(&bar_ap);
-            issue_mma(tbase + TM_C, sb + OFF_KQ, 16384, false, 0, sb + OFF_SB, 0, true, 16384, 8, ID_KxMN, false);
+            issue_mma<8, false, 16384, true, 16384>(tbase + TM_C, sb + OFF_KQ, sb + OFF_SB, ID_KxMN, false);
             mma_commit(&bar_c);
         }
 
-        // ================= step 3: P and A from TMEM, Kb tile =================
+        // ================= step 3: P and A from TMEM; Kb tile; diagonal blocks of (I+A)^-1 =========
         ok = mbar_wait(&bar_ap, par, kTimeoutNs);
         tc_fence_after_sync();
         ok = __syncthreads_and(ok) != 0;
         if (!ok) break;
-        {
-            // Kb (MN-major A of MMA6: row = token j, column = channel i)
+        float* AF = reinterpret_cast<float*>(sm + OFF_AF);   // A, fp32, row stride kLd
+        float* XF = reinterpret_cast<float*>(sm + OFF_X);    // X = (I+A)^-1, row-major
+        float* XT = reinterpret_cast<float*>(sm + OFF_XT);   // X transposed
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const uint16_t bits = (uint16_t)((kb_pack[j >> 1] >> ((j & 1) * 16)) & 0xFFFFu);
-                *reinterpret_cast<uint16_t*>(sm + OFF_KBAR + sw128_offset(32 * hf + j, (uint32_t)ci, 8192)) = bits;
-            }
-        }
+        for (int g8 = 0; g8 < 4; ++g8)
+            *reinterpret_cast<uint4*>(sm + OFF_KBAR + sw128_offset(tr, c0 + 8 * g8, 8192)) =
+                make_uint4(kb[4 * g8], kb[4 * g8 + 1], kb[4 * g8 + 2], kb[4 * g8 + 3]);
         if (warp < 4) {
             // lane L of TM_AP: L < 32: Qt0 row r = L; L < 64: Kt0 row r = L - 32;
             //                  L < 96: Qt1 row r = L - 32; else Kt1 row r = L - 64.
             const int L = 32 * warp + lane;
-            const bool is_q = (L < 32) || (L >= 64 && L < 96);
+            const bool is_q = (warp == 0) || (warp == 2);
             const int r = (L < 64) ? (L & 31) : 32 + (L & 31);
             float row[64];
-            if (r < 32) {
+            if (warp < 2) {
 #pragma unroll
                 for (int cb = 0; cb < 32; cb += 16) tmem_ld16(tlane + TM_AP + cb, row + cb);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 32; j < 64; ++j) row[j] = 0.f;
             } else {
-                float dg[32];
-                // MMA2 columns 0..31 hold the off-diagonal block (cols j = 0..31)
+                // MMA2 columns 0..31: off-diagonal block (j = 0..31); MMA1 columns 32..63: block 1 (j = 32..63)
 #pragma unroll
                 for (int cb = 0; cb < 32; cb += 16) tmem_ld16(tlane + TM_AP + 64 + cb, row + cb);
-                // MMA1 columns 32..63 hold the diagonal block of block 1 (cols j = 32..63)
 #pragma unroll
-                for (int cb = 0; cb < 32; cb += 16) tmem_ld16(tlane + TM_AP + 32 + cb, dg + cb);
+                for (int cb = 0; cb < 32; cb += 16) tmem_ld16(tlane + TM_AP + 32 + cb, row + 32 + cb);
                 tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) row[32 + j] = dg[j];
             }
             if (is_q) {
-                // P row r: lower triangle including the diagonal, bf16, K-major rows 64.. of the P tile
+                // P row r: lower triangle including the diagonal, bf16, rows 64.. of the P tile
 #pragma unroll
                 for (int j = 0; j < 64; j += 8) {
-                    uint4 pk;
                     float v8[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) v8[e] = (j + e <= r) ? row[j + e] : 0.f;
-                    pk.x = pack_bf16x2(v8[0], v8[1]); pk.y = pack_bf16x2(v8[2], v8[3]);
-                    pk.z = pack_bf16x2(v8[4], v8[5]); pk.w = pack_bf16x2(v8[6], v8[7]);
-                    *reinterpret_cast<uint4*>(sm + OFF_PV + 8192 + sw128_offset(r, j, 8192)) = pk;
+                    *reinterpret_cast<uint4*>(sm + OFF_PV + 8192 + sw128_offset(r, j, 8192)) =
+                        make_uint4(pack_bf16x2(v8[0], v8[1]), pack_bf16x2(v8[2], v8[3]),
+                                   pack_bf16x2(v8[4], v8[5]), pack_bf16x2(v8[6], v8[7]));
                 }
             } else {
-                // A row r: strictly lower, scaled by beta_r, fp32 row-major for the solve
+                // A row r: strictly lower, scaled by beta_r (select first: masked entries may be inf)
                 const float br = s_beta[r];
-                float* arow = reinterpret_cast<float*>(sm + OFF_AF) + r * 64;
 #pragma unroll
-                for (int j = 0; j < 64; j += 4) {
-                    float4 w;
-                    w.x = (j + 0 < r) ? br * row[j + 0] : 0.f;
-                    w.y = (j + 1 < r) ? br * row[j + 1] : 0.f;
-                    w.z = (j + 2 < r) ? br * row[j + 2] : 0.f;
-                    w.w = (j + 3 < r) ? br * row[j + 3] : 0.f;
-                    *reinterpret_cast<float4*>(arow + j) = w;
+                for (int j = 0; j < 64; ++j) row[j] = (j < r) ? br * row[j] : 0.f;
+#pragma unroll
+                for (int j = 0; j < 64; j += 4)
+                    *reinterpret_cast<float4*>(AF + r * kLd + j) = make_float4(row[j], row[j + 1], row[j + 2], row[j + 3]);
+                // diagonal 16x16 block of X = (I + A)^-1 by forward substitution across the
+                // 16 lanes that own its rows (two blocks per warp, one per half-warp)
+                const int s16 = r & 15, blk = r >> 4, base = lane & 16;
+                float dg[16];
+                if (warp == 1) {
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) dg[t] = (lane < 16) ? row[t] : row[16 + t];
+                } else {
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) dg[t] = (lane < 16) ? row[32 + t] : row[48 + t];
                 }
+                float x[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) x[c] = (c == s16) ? 1.f : 0.f;
+#pragma unroll
+                for (int t = 0; t < 15; ++t) {
+                    float xt[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) xt[c] = __shfl_sync(0xffffffffu, x[c], base + t);
+                    if (s16 > t) {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) x[c] = fmaf(-dg[t], xt[c], x[c]);
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < 16; c += 4)
+                    *reinterpret_cast<float4*>(XF + r * kLd + 16 * blk + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) XT[(16 * blk + c) * kLd + r] = x[c];
             }
         }
         __syncthreads();
 
-        // ================= step 4: X = (I + A)^{-1} (fp32, 16x16 blocks), T = X Diag(beta) ==========
+        // ================= step 4: off-diagonal blocks of X, then T = X Diag(beta) ================
+        // X_RJ = -X_RR sum_{L=J}^{R-1} A_RL X_LJ, by block distance d = R - J (16x16 blocks), on
+        // warp-level bf16 tensor-core tiles with fp32 accumulation (the chunk model shows bf16
+        // operands here leave the output error unchanged).  Warp 2*qb + nt computes the 8 output
+        // columns nt of block qb of the level.
         {
-            const float* Am = reinterpret_cast<const float*>(sm + OFF_AF);
-            float* X = reinterpret_cast<float*>(sm + OFF_X);
-            float* W = reinterpret_cast<float*>(sm + OFF_W);
-            // diagonal blocks by forward substitution, one thread per (block, column)
-            if (tid < 64) {
-                const int bb = tid >> 4, c = tid & 15, o0 = 16 * bb;
-                float x[16];
+            const int g4 = lane >> 2, t4 = lane & 3;
+            float* WS = reinterpret_cast<float*>(sm + OFF_WS) + warp * 8 * kLdS;  // this warp's W^T (8 x 16)
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    float s = (rr == c) ? 1.f : 0.f;
-#pragma unroll
-                    for (int l = 0; l < rr; ++l) s -= Am[(o0 + rr) * 64 + o0 + l] * x[l];
-                    x[rr] = (rr < c) ? 0.f : s;
-                }
-#pragma unroll
-                for (int rr = 0; rr < 16; ++rr) X[(o0 + rr) * 64 + o0 + c] = x[rr];
-            } else if (tid < 128) {
-                // zero the strictly upper blocks of X
-                const int t = tid - 64;
-                for (int e = t; e < 64 * 64; e += 64) {
-                    const int rr = e >> 6, cc = e & 63;
-                    if ((cc >> 4) > (rr >> 4)) X[e] = 0.f;
-                }
-            }
-            __syncthreads();
-            // off-diagonal blocks, by distance d = R - J: X_RJ = -X_RR sum_{L=J}^{R-1} A_RL X_LJ
-            const int er = tid >> 4, ec = tid & 15;
-#pragma unroll 1
             for (int d = 1; d < 4; ++d) {
-                const int nblk = 4 - d;
-                for (int q = 0; q < nblk; ++q) {
-                    const int R = q + d, J = q;
-                    float s = 0.f;
-                    for (int L = J; L < R; ++L)
+                if (warp < 2 * (4 - d)) {
+                    const int qb = warp >> 1, nt = warp & 1;
+                    const int R = qb + d, J = qb;
+                    float w[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                        for (int l = 0; l < 16; ++l)
-                            s += Am[(16 * R + er) * 64 + 16 * L + l] * X[(16 * L + l) * 64 + 16 * J + ec];
-                    W[q * 256 + er * 16 + ec] = s;
-                }
-                __syncthreads();
-                for (int q = 0; q < nblk; ++q) {
-                    const int R = q + d, J = q;
-                    float s = 0.f;
-#pragma unroll
-                    for (int l = 0; l < 16; ++l) s -= X[(16 * R + er) * 64 + 16 * R + l] * W[q * 256 + l * 16 + ec];
-                    X[(16 * R + er) * 64 + 16 * J + ec] = s;
+                    for (int Lb = 0; Lb < 3; ++Lb) {
+                        if (Lb < d) {
+                            const int L = J + Lb;
+                            uint32_t af[4], bf[2];
+                            load_a_frag(AF + (16 * R) * kLd + 16 * L, kLd, g4, t4, af);
+                            load_b_frag(XT + (16 * J + 8 * nt) * kLd + 16 * L, kLd, g4, t4, bf);
+                            mma_16816(w, af, bf);
+                        }
+                    }
+                    // W (16 x 8, this warp's columns) -> transposed scratch, read back as the B fragment
+                    WS[(2 * t4) * kLdS + g4] = w[0];
+                    WS[(2 * t4 + 1) * kLdS + g4] = w[1];
+                    WS[(2 * t4) * kLdS + g4 + 8] = w[2];
+                    WS[(2 * t4 + 1) * kLdS + g4 + 8] = w[3];
+                    __syncwarp();
+                    uint32_t af[4], bf[2];
+                    load_a_frag(XF + (16 * R) * kLd + 16 * R, kLd, g4, t4, af);
+                    load_b_frag(WS, kLdS, g4, t4, bf);
+                    float x[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma_16816(x, af, bf);
+                    const int col = 16 * J + 8 * nt + 2 * t4;
+                    *reinterpret_cast<float2*>(XF + (16 * R + g4) * kLd + col) = make_float2(-x[0], -x[1]);
+                    *reinterpret_cast<float2*>(XF + (16 * R + g4 + 8) * kLd + col) = make_float2(-x[2], -x[3]);
+                    XT[col * kLd + 16 * R + g4] = -x[0];
+                    XT[(col + 1) * kLd + 16 * R + g4] = -x[1];
+                    XT[col * kLd + 16 * R + g4 + 8] = -x[2];
+                    XT[(col + 1) * kLd + 16 * R + g4 + 8] = -x[3];
                 }
                 __syncthreads();
             }
-            // T = X Diag(beta) -> bf16 K-major tile rows 0..63 (K = 64 tokens)
+            // T = X Diag(beta) -> bf16 K-major tile rows 0..63 (K = 64 tokens); upper blocks are 0
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int idx = tid + kThreads * e;  // 512 chunks of 8
                 const int r = idx >> 3, j = (idx & 7) * 8;
-                const float* xr = X + r * 64 + j;
-                uint4 pk;
-                pk.x = pack_bf16x2(xr[0] * s_beta[j + 0], xr[1] * s_beta[j + 1]);
-                pk.y = pack_bf16x2(xr[2] * s_beta[j + 2], xr[3] * s_beta[j + 3]);
-                pk.z = pack_bf16x2(xr[4] * s_beta[j + 4], xr[5] * s_beta[j + 5]);
-                pk.w = pack_bf16x2(xr[6] * s_beta[j + 6], xr[7] * s_beta[j + 7]);
+                uint4 pk = make_uint4(0u, 0u, 0u, 0u);
+                if ((j >> 4) <= (r >> 4)) {
+                    const float4 xa = *reinterpret_cast<const float4*>(XF + r * kLd + j);
+                    const float4 xb = *reinterpret_cast<const float4*>(XF + r * kLd + j + 4);
+                    pk.x = pack_bf16x2(xa.x * s_beta[j + 0], xa.y * s_beta[j + 1]);
+                    pk.y = pack_bf16x2(xa.z * s_beta[j + 2], xa.w * s_beta[j + 3]);
+                    pk.z = pack_bf16x2(xb.x * s_beta[j + 4], xb.y * s_beta[j + 5]);
+                    pk.w = pack_bf16x2(xb.z * s_beta[j + 6], xb.w * s_beta[j + 7]);
+                }
                 *reinterpret_cast<uint4*>(sm + OFF_T + sw128_offset(r, j, 8192)) = pk;
             }
         }
@@ -435,25 +564,22 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (!ok) break;
         if (quarter < 2) {
             const int r = 32 * quarter + lane;
+            float ks[64];
 #pragma unroll
-            for (int cb = 0; cb < 64; cb += 16) {
-                const int c0 = 64 * colhalf + cb;
-                float ks[16];
-                tmem_ld16(tlane + TM_C + c0, ks);
-                tmem_wait_ld();
+            for (int cb = 0; cb < 64; cb += 16) tmem_ld16(tlane + TM_C + 64 * colhalf + cb, ks + cb);
+            tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; j += 8) {
-                    const uint32_t off = sw128_offset(r, c0 + j, 8192);
-                    const uint4 vv = *reinterpret_cast<const uint4*>(sm + OFF_RAW_V + off);
-                    const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vv);
-                    uint4 pk;
-                    float2 f;
-                    f = __bfloat1622float2(v2[0]); pk.x = pack_bf16x2(f.x - ks[j + 0], f.y - ks[j + 1]);
-                    f = __bfloat1622float2(v2[1]); pk.y = pack_bf16x2(f.x - ks[j + 2], f.y - ks[j + 3]);
-                    f = __bfloat1622float2(v2[2]); pk.z = pack_bf16x2(f.x - ks[j + 4], f.y - ks[j + 5]);
-                    f = __bfloat1622float2(v2[3]); pk.w = pack_bf16x2(f.x - ks[j + 6], f.y - ks[j + 7]);
-                    *reinterpret_cast<uint4*>(sm + OFF_YU + off) = pk;
-                }
+            for (int j = 0; j < 64; j += 8) {
+                const uint32_t off = sw128_offset(r, 64 * colhalf + j, 8192);
+                const uint4 vv = *reinterpret_cast<const uint4*>(sm + OFF_RAW_V + off);
+                const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vv);
+                uint4 pk;
+                float2 f;
+                f = __bfloat1622float2(v2[0]); pk.x = pack_bf16x2(f.x - ks[j + 0], f.y - ks[j + 1]);
+                f = __bfloat1622float2(v2[1]); pk.y = pack_bf16x2(f.x - ks[j + 2], f.y - ks[j + 3]);
+                f = __bfloat1622float2(v2[2]); pk.z = pack_bf16x2(f.x - ks[j + 4], f.y - ks[j + 5]);
+                f = __bfloat1622float2(v2[3]); pk.w = pack_bf16x2(f.x - ks[j + 6], f.y - ks[j + 7]);
+                *reinterpret_cast<uint4*>(sm + OFF_YU + off) = pk;
             }
         }
         fence_proxy_async_smem();
@@ -466,23 +592,21 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 issue_loads(chunk + 1);
                 pending_chunk = chunk + 1;
             }
-            issue_mma(tbase + TM_U, sb + OFF_T, 0, false, 0, sb + OFF_YU, 0, true, 8192, 4, ID_KxMN, false);
+            issue_mma<4, false, 0, true, 8192>(tbase + TM_U, sb + OFF_T, sb + OFF_YU, ID_KxMN, false);
             mma_commit(&bar_u);
         }
 
         // ================= step 7: decay the fp32 state in TMEM; U -> bf16 tile =================
         {
+            float sv[64];
 #pragma unroll
-            for (int cb = 0; cb < 64; cb += 16) {
-                const int c0 = 64 * colhalf + cb;
-                float sv[16];
-                tmem_ld16(tlane + TM_S + c0, sv);
-                tmem_wait_ld();
-                const float gc = s_gammaC[32 * quarter + lane];
+            for (int cb = 0; cb < 64; cb += 16) tmem_ld16(tlane + TM_S + 64 * colhalf + cb, sv + cb);
+            tmem_wait_ld();
+            const float gc = s_gammaC[32 * quarter + lane];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) sv[j] *= gc;
-                tmem_st16(tlane + TM_S + c0, sv);
-            }
+            for (int j = 0; j < 64; ++j) sv[j] *= gc;
+#pragma unroll
+            for (int cb = 0; cb < 64; cb += 16) tmem_st16(tlane + TM_S + 64 * colhalf + cb, sv + cb);
             tmem_wait_st();
         }
         ok = mbar_wait(&bar_u, par, kTimeoutNs);
@@ -491,20 +615,15 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (!ok) break;
         if (quarter < 2) {
             const int r = 32 * quarter + lane;
+            float u[64];
 #pragma unroll
-            for (int cb = 0; cb < 64; cb += 16) {
-                const int c0 = 64 * colhalf + cb;
-                float u[16];
-                tmem_ld16(tlane + TM_U + c0, u);
-                tmem_wait_ld();
+            for (int cb = 0; cb < 64; cb += 16) tmem_ld16(tlane + TM_U + 64 * colhalf + cb, u + cb);
+            tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; j += 8) {
-                    uint4 pk;
-                    pk.x = pack_bf16x2(u[j], u[j + 1]); pk.y = pack_bf16x2(u[j + 2], u[j + 3]);
-                    pk.z = pack_bf16x2(u[j + 4], u[j + 5]); pk.w = pack_bf16x2(u[j + 6], u[j + 7]);
-                    *reinterpret_cast<uint4*>(sm + OFF_YU + sw128_offset(r, c0 + j, 8192)) = pk;
-                }
-            }
+            for (int j = 0; j < 64; j += 8)
+                *reinterpret_cast<uint4*>(sm + OFF_YU + sw128_offset(r, 64 * colhalf + j, 8192)) =
+                    make_uint4(pack_bf16x2(u[j], u[j + 1]), pack_bf16x2(u[j + 2], u[j + 3]),
+                               pack_bf16x2(u[j + 4], u[j + 5]), pack_bf16x2(u[j + 6], u[j + 7]));
         }
         fence_proxy_async_smem();
         tc_fence_before_sync();
@@ -512,8 +631,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (tid == 0) {
             tc_fence_after_sync();
             // O = Qt S + P U (onto lanes 64..127 of TM_C); S <- Diag(gamma_C) S + Kb^T U
-            issue_mma(tbase + TM_C, sb + OFF_PV, 0, false, 0, sb + OFF_YU, 0, true, 8192, 4, ID_KxMN, true);
-            issue_mma(tbase + TM_S, sb + OFF_KBAR, 0, true, 8192, sb + OFF_YU, 0, true, 8192, 4, ID_MNxMN, true);
+            issue_mma<4, false, 0, true, 8192>(tbase + TM_C, sb + OFF_PV, sb + OFF_YU, ID_KxMN, true);
+            issue_mma<4, true, 8192, true, 8192>(tbase + TM_S, sb + OFF_KBAR, sb + OFF_YU, ID_MNxMN, true);
             mma_commit(&bar_os);
         }
 
@@ -525,41 +644,29 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (quarter >= 2) {
             const int r = 32 * (quarter - 2) + lane;
             // tcgen05.ld is warp-collective: every lane loads, only valid tokens are stored
-            const bool valid = r < nvalid;
-            __nv_bfloat16* orow = p.o + (((size_t)b * T + t0 + (valid ? r : 0)) * p.H + h) * kD;
+            float ov[64];
 #pragma unroll
-            for (int cb = 0; cb < 64; cb += 16) {
-                const int c0 = 64 * colhalf + cb;
-                float ov[16];
-                tmem_ld16(tlane + TM_C + c0, ov);
-                tmem_wait_ld();
-                if (valid) {
-                    uint4 pk0, pk1;
-                    pk0.x = pack_bf16x2(ov[0], ov[1]); pk0.y = pack_bf16x2(ov[2], ov[3]);
-                    pk0.z = pack_bf16x2(ov[4], ov[5]); pk0.w = pack_bf16x2(ov[6], ov[7]);
-                    pk1.x = pack_bf16x2(ov[8], ov[9]); pk1.y = pack_bf16x2(ov[10], ov[11]);
-                    pk1.z = pack_bf16x2(ov[12], ov[13]); pk1.w = pack_bf16x2(ov[14], ov[15]);
-                    *reinterpret_cast<uint4*>(orow + c0) = pk0;
-                    *reinterpret_cast<uint4*>(orow + c0 + 8) = pk1;
-                }
+            for (int cb = 0; cb < 64; cb += 16) tmem_ld16(tlane + TM_C + 64 * colhalf + cb, ov + cb);
+            tmem_wait_ld();
+            if (r < nvalid) {
+                uint4* orow = reinterpret_cast<uint4*>(p.o + (((size_t)b * T + t0 + r) * p.H + h) * kD + 64 * colhalf);
+#pragma unroll
+                for (int j = 0; j < 64; j += 8)
+                    orow[j >> 3] = make_uint4(pack_bf16x2(ov[j], ov[j + 1]), pack_bf16x2(ov[j + 2], ov[j + 3]),
+                                              pack_bf16x2(ov[j + 4], ov[j + 5]), pack_bf16x2(ov[j + 6], ov[j + 7]));
             }
         }
         {
             const int i = 32 * quarter + lane;
+            float sv[64];
 #pragma unroll
-            for (int cb = 0; cb < 64; cb += 16) {
-                const int c0 = 64 * colhalf + cb;
-                float sv[16];
-                tmem_ld16(tlane + TM_S + c0, sv);
-                tmem_wait_ld();
+            for (int cb = 0; cb < 64; cb += 16) tmem_ld16(tlane + TM_S + 64 * colhalf + cb, sv + cb);
+            tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; j += 8) {
-                    uint4 pk;
-                    pk.x = pack_bf16x2(sv[j], sv[j + 1]); pk.y = pack_bf16x2(sv[j + 2], sv[j + 3]);
-                    pk.z = pack_bf16x2(sv[j + 4], sv[j + 5]); pk.w = pack_bf16x2(sv[j + 6], sv[j + 7]);
-                    *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_offset(i, c0 + j, 16384)) = pk;
-                }
-            }
+            for (int j = 0; j < 64; j += 8)
+                *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_offset(i, 64 * colhalf + j, 16384)) =
+                    make_uint4(pack_bf16x2(sv[j], sv[j + 1]), pack_bf16x2(sv[j + 2], sv[j + 3]),
+                               pack_bf16x2(sv[j + 4], sv[j + 5]), pack_bf16x2(sv[j + 6], sv[j + 7]));
         }
         fence_proxy_async_smem();
         tc_fence_before_sync();
