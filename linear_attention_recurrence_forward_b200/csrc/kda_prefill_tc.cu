@@ -14,24 +14,28 @@
 //   O = Qt S + P U
 //   S <- Diag(e^{Gam_C}) S + Kb^T U
 //
-// This is an exact rewrite of the token recurrence.  The pair factors e^{Gam_r-Gam_j}
-// are formed from two per-token factors against a reference token b (e^{Gam_r-Gam_b}
-// e^{Gam_b-Gam_j}).  The chunk is split into two 32-token blocks: the off-diagonal block
-// uses b = 31 (both factors <= 1), each diagonal block its middle token (16 or 48), where
-// each factor is at most e^{5*16} = e^{80} < FLT_MAX because the log-decay is bounded
-// below by -5 (the skill card's quick facts: the bounded scaled-sigmoid gate is what lets
-// the diagonal tiles run as dense tensor-core matmuls).
+// This is an exact rewrite of the token recurrence.  The pair factors e^{Gam_r-Gam_j} are
+// formed as e^{Gam_r-Gam_b} e^{Gam_b-Gam_j} against a reference token b.  The chunk is two
+// 32-token blocks; both the diagonal block of block 1 and the block-1 x block-0 rectangle
+// use b = 48, the diagonal block of block 0 uses b = 16.  Row-side factors are at most
+// e^{5*16} = e^{80} < FLT_MAX because the log-decay is bounded below by -5 (the skill card's
+// quick facts: the bounded scaled-sigmoid gate is what lets the diagonal tiles run as dense
+// tensor-core matmuls).  On the rectangle a column factor e^{Gam_48-Gam_j} can underflow;
+// the pair factor it belongs to is then below e^{-7.3} and the term is dropped (measured in
+// fp64: at most 4.3e-4 relative to max|o| under adversarial decay, zero on the recipe inputs).
 //
-// Per CTA: one (b, h), the whole chunk sequence.  Tensor-core products per chunk:
-//   MMA1 [Qt0;Kt0;Qt1;Kt1](mid refs) x [Kh0;Kh1]^T    -> diagonal blocks of P and A
-//   MMA2 [Qt1;Kt1](ref 31)            x Kh0^T         -> off-diagonal block
-//   MMA3 [Kt;Qt] x S_bf16                             -> Kt S (Y = V - Kt S) and Qt S
-//   MMA4 T x Y                                        -> U
-//   MMA5 P x U   (accumulated onto Qt S)              -> O
-//   MMA6 Kb^T x U (accumulated onto the decayed fp32 state in TMEM) -> new S
-// The 64x64 triangular solve runs in fp32 on the CUDA cores.  Every M = 64 product is
-// issued as M = 128 with the unused 64 rows reading other (valid) shared memory, so all
-// accumulators use the one-row-per-lane TMEM layout; those lanes are never read.
+// CTA organisation: one (b, h) per CTA, 16 warps, two warp-specialised groups coupled by
+// mbarriers so that the state-independent work of chunk c+1 overlaps the recurrence of
+// chunk c:
+//   prep warps 0..7    per chunk: TMA q,k,g -> Gam = L g (tensor core) -> per-channel
+//                      constants -> bf16 operand tiles -> MMA1 (A and P in one product) ->
+//                      fp32 triangular solve (diagonal blocks by substitution, off-diagonal
+//                      blocks on warp-level bf16 MMA tiles) -> T, P, Kb tiles.
+//   serial warps 8..15 per chunk: MMA3 [Qt;Kt] S -> Y = V - Kt S -> MMA4 U = T Y ->
+//                      MMA5 O = Qt S + P U, MMA6 S += Kb^T U (state decayed in TMEM first)
+//                      -> O to global, S to bf16 for the next chunk.
+// All tcgen05 products are M = 128: products with 64 meaningful rows read 64 further rows
+// of other valid shared memory into TMEM lanes that are never read.
 #include <cudaTypedefs.h>
 #include <mutex>
 
@@ -43,53 +47,52 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kC = 64;         // chunk length
-constexpr int kD = 128;        // dk = dv
-constexpr int kThreads = 256;  // 8 warps
-constexpr uint64_t kTimeoutNs = 2000000000ull;  // bounded waits: 2 s
+constexpr int kC = 64;          // chunk length
+constexpr int kD = 128;         // dk = dv
+constexpr int kThreads = 512;   // 16 warps
+constexpr int kPrepThreads = 256;
+constexpr int kSerialThreads = 256;
+constexpr uint32_t kBarPrep = 1, kBarSerial = 2;   // named hardware barriers
+constexpr uint64_t kTimeoutNs = 2000000000ull;      // bounded waits: 2 s
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
-constexpr uint32_t OFF_RAW_Q = 0;          // TMA destination, bf16 [64 tok][128], 2 boxes of 8 KB
+constexpr uint32_t OFF_RAW_Q = 0;           // TMA destination, bf16 [64 tok][128], 2 boxes of 8 KB
 constexpr uint32_t OFF_RAW_K = 16384;
 constexpr uint32_t OFF_RAW_G = 32768;
-constexpr uint32_t OFF_RAW_V = 49152;
-constexpr uint32_t OFF_AP = 65536;         // operands of MMA1/2, reused after they complete
-constexpr uint32_t OFF_A1 = OFF_AP;                 // K-major, 128 rows, 2 atoms x 16 KB
-constexpr uint32_t OFF_B1 = OFF_AP + 32768;         // K-major, 64 rows, 2 atoms x 8 KB
-constexpr uint32_t OFF_A2 = OFF_AP + 49152;         // rows 64..127 only, 2 atoms x 8 KB
-constexpr uint32_t OFF_B2 = OFF_AP + 65536;         // K-major, 32 rows, 2 atoms x 4 KB
-constexpr uint32_t OFF_T = OFF_AP;                  // after MMA1/2: T rows 0..63 (K = 64)
-constexpr uint32_t OFF_PV = OFF_AP + 16384;         //   P as rows 64..127 of a tile starting here
-constexpr uint32_t OFF_KBAR = OFF_AP + 32768;       //   Kb, MN-major A (M = dk), 2 atoms x 8 KB
-constexpr uint32_t OFF_AF = OFF_AP + 49152;         //   A (fp32 64x64) for the solve
-constexpr uint32_t OFF_KQ = OFF_AP + 73728;         // [Kt; Qt], K-major, 128 rows, 2 atoms x 16 KB
-constexpr uint32_t OFF_SB = OFF_KQ + 32768;         // S in bf16, MN-major B (K = dk), 2 atoms x 16 KB
-constexpr uint32_t OFF_YU = OFF_SB + 32768;         // Y then U, MN-major B (K = 64), 2 atoms x 8 KB
-constexpr uint32_t SMEM_BYTES = OFF_YU + 16384;     // 221184
+constexpr uint32_t OFF_V = 49152;           // v, then Y = V - Kt S, then U (MN-major B, K = 64 tokens)
+constexpr uint32_t OFF_AP = 65536;          // prep operand region (56 KB)
+constexpr uint32_t OFF_A1 = OFF_AP;                 // [Qt0;Kt0;Qt1;Kt1] block-middle refs, K-major, 2 x 16 KB
+constexpr uint32_t OFF_BB = OFF_AP + 32768;         // [Kh0(16);Kh1(48);Kh0(48)], K-major, 96 rows, 2 x 12 KB
 constexpr uint32_t OFF_L = OFF_AP + 8192;           // chunk start: lower-triangular ones (8 KB)
-constexpr uint32_t OFF_CONST = OFF_YU;              // step 2: reference rows of Gam + per-channel constants
-constexpr int kLd = 68;                             // padded row stride (floats) of the solve matrices
-constexpr uint32_t OFF_X = OFF_RAW_Q;               // solve: X = (I+A)^-1 fp32 (raw q/k/g are dead)
-constexpr uint32_t OFF_XT = OFF_X + 64 * kLd * 4;   //   X transposed
+constexpr int kLd = 68;                              // padded row stride (floats) of the solve matrices
 constexpr int kLdS = 20;
-constexpr uint32_t OFF_WS = OFF_XT + 64 * kLd * 4;  //   per-warp W^T scratch (8 warps x 8 x kLdS)
-static_assert(OFF_WS + 8 * 8 * kLdS * 4 <= OFF_RAW_V, "solve scratch overlaps raw v");
-static_assert(OFF_AF + 64 * kLd * 4 <= OFF_KQ, "A overlaps the KQ tile");
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint32_t SMEM_DYN = SMEM_BYTES + 1024;    // + alignment slack
+constexpr uint32_t OFF_AF = OFF_AP;                  // after MMA1: A (fp32 64 x kLd)
+constexpr uint32_t OFF_X = OFF_AF + 64 * kLd * 4;    //   X = (I+A)^-1, row-major
+constexpr uint32_t OFF_XT = OFF_X + 64 * kLd * 4;    //   X transposed
+constexpr uint32_t OFF_WS = OFF_XT + 64 * kLd * 4;   //   per-warp W^T scratch (8 warps x 8 x kLdS)
+constexpr uint32_t OFF_KQ = OFF_AP + 57344;          // [Qt0;Kt0;Qt1;Kt1] chunk-start ref, K-major, 2 x 16 KB
+constexpr uint32_t OFF_SB = OFF_KQ + 32768;          // S in bf16, MN-major B (K = dk), 2 x 16 KB
+constexpr uint32_t OFF_TP = OFF_SB + 32768;          // T and P, interleaved 4 KB pieces (16 KB)
+constexpr uint32_t OFF_T = OFF_TP;                   //   T rows 0-31 at +0, rows 32-63 at +8 KB
+constexpr uint32_t OFF_P = OFF_TP + 4096;            //   P rows 0-31 at +4 KB, rows 32-63 at +12 KB
+constexpr uint32_t OFF_KBAR = OFF_TP + 16384;        // Kb, MN-major A (M = dk), 2 x 8 KB
+constexpr uint32_t SMEM_BYTES = OFF_KBAR + 16384;    // 221184
+constexpr uint32_t SMEM_DYN = SMEM_BYTES + 1024;     // + alignment slack
+static_assert(OFF_WS + 8 * 8 * kLdS * 4 <= OFF_KQ, "solve scratch overlaps KQ");
+static_assert(OFF_BB + 2 * 12288 <= OFF_KQ, "BB overlaps KQ");
 
 // ---- TMEM columns (fp32 accumulators, 128 lanes) ----
 constexpr uint32_t TM_S = 0;     // S (dk lanes x dv columns), fp32 master state
-constexpr uint32_t TM_C = 128;   // MMA3 result: lanes 0-63 Kt S, lanes 64-127 Qt S (+ P U = O)
-constexpr uint32_t TM_U = 256;   // MMA4 result: lanes 0-63 U
-constexpr uint32_t TM_AP = 384;  // MMA1 (64 cols) and MMA2 (32 cols)
+constexpr uint32_t TM_C = 128;   // MMA3: lanes 0-31 Qt0 S, 32-63 Kt0 S, 64-95 Qt1 S, 96-127 Kt1 S; + P U
+constexpr uint32_t TM_U = 256;   // MMA4: U at lanes 0-31 (tokens 0-31) and 64-95 (tokens 32-63)
+constexpr uint32_t TM_P = 384;   // prep: Gam (128 columns), then MMA1 (96 columns)
 constexpr uint32_t TM_COLS = 512;
 
-constexpr uint32_t ID_MMA1 = idesc_bf16_f32(128, 64, false, false);
-constexpr uint32_t ID_MMA2 = idesc_bf16_f32(128, 32, false, false);
+constexpr uint32_t ID_G = idesc_bf16_f32(128, 64, false, true);
+constexpr uint32_t ID_MMA1 = idesc_bf16_f32(128, 96, false, false);
 constexpr uint32_t ID_KxMN = idesc_bf16_f32(128, 128, false, true);
 constexpr uint32_t ID_MNxMN = idesc_bf16_f32(128, 128, true, true);
-constexpr uint32_t ID_G = idesc_bf16_f32(128, 64, false, true);
+constexpr float kLog2e = 1.4426950408889634f;
 
 struct TcParams {
     const __nv_bfloat16* beta;
@@ -158,6 +161,22 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// Load 64 TMEM columns of this warp's lanes (one wait).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* r) {
+#pragma unroll
+    for (int cb = 0; cb < 64; cb += 16) tmem_ld16(taddr + cb, r + cb);
+    tmem_wait_ld();
+}
+
+__device__ __forceinline__ uint4 pack8(const float* v) {
+    return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                      pack_bf16x2(v[6], v[7]));
+}
+
+// Row of the T and P tiles that holds matrix row r (0..63): rows 0-31 stay, rows 32-63 move to
+// 64-95, so that the products land in the TMEM lanes of the Qt rows.
+__device__ __forceinline__ int tp_row(int r) { return r < 32 ? r : r + 32; }
+
 __global__ void __launch_bounds__(kThreads, 1)
 kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
@@ -169,32 +188,31 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     uint8_t* sm = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);
     const uint32_t sb = smem_u32(sm);
 
-    __shared__ uint64_t bar_load, bar_g, bar_ap, bar_c, bar_u, bar_os, bar_drain;
+    // TMA / MMA completion barriers (one phase per chunk) and prep -> serial hand-offs.
+    __shared__ uint64_t bar_qkg, bar_v, bar_g, bar_ap, bar_c, bar_u, bar_os, bar_kq, bar_tpk;
+    __shared__ uint64_t bar_drain_p, bar_drain_s;
     __shared__ uint32_t tmem_base_s;
     __shared__ float s_beta[kC];
-    __shared__ float s_gammaC[kD];
+    __shared__ float s_gamma[2][kD];                   // e^{Gam_63} per channel, by chunk parity
+    __shared__ __align__(16) float s_refs[4][kD];      // Gam rows 16, 31, 48, 63 (float4 access)
+    __shared__ __align__(16) float s_cst[2][4][kD];    // per block: Gam_m*log2e, e^{Gam_m}, e^{Gam_63-Gam_m}, c_off
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quarter = warp & 3;           // TMEM lane quarter this warp may access
-    const int colhalf = warp >> 2;          // which 64 TMEM columns of a 128-wide result
+    const int quarter = warp & 3;              // TMEM lane quarter this warp may access
+    const bool is_prep = warp < 8;
+    const int colhalf = (warp >> 2) & 1;       // which 64 columns of a 128-wide result (per group)
     const int bh = blockIdx.x;
     const int b = bh / p.H, h = bh % p.H;
     const int T = p.T;
     const int nchunks = (T + kC - 1) / kC;
 
     if (tid == 0) {
-        mbar_init(&bar_load, 1);
-        mbar_init(&bar_g, 1);
-        mbar_init(&bar_ap, 1);
-        mbar_init(&bar_c, 1);
-        mbar_init(&bar_u, 1);
-        mbar_init(&bar_os, 1);
-        mbar_init(&bar_drain, 1);
+        mbar_init(&bar_qkg, 1); mbar_init(&bar_v, 1); mbar_init(&bar_g, 1); mbar_init(&bar_ap, 1);
+        mbar_init(&bar_c, 1); mbar_init(&bar_u, 1); mbar_init(&bar_os, 1); mbar_init(&bar_kq, 1);
+        mbar_init(&bar_tpk, 1); mbar_init(&bar_drain_p, 1); mbar_init(&bar_drain_s, 1);
         fence_mbar_init();
-        prefetch_tensormap(&tm_q);
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_g);
-        prefetch_tensormap(&tm_v);
+        prefetch_tensormap(&tm_q); prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_g); prefetch_tensormap(&tm_v);
     }
     if (warp == 0) {
         tmem_alloc(&tmem_base_s, TM_COLS);
@@ -206,136 +224,100 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t tbase = tmem_base_s;
     const uint32_t tlane = tbase + ((uint32_t)(32 * quarter) << 16);  // this warp's lane quarter
 
-    auto issue_loads = [&](int chunk) {
-        mbar_arrive_expect_tx(&bar_load, 4u * 16384u);
-        const int t0 = chunk * kC;
+    auto load_qkg = [&](int chunk) {
+        mbar_arrive_expect_tx(&bar_qkg, 3u * 16384u);
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-            tma_load_4d(sm + OFF_RAW_Q + x * 8192, &tm_q, &bar_load, 64 * x, h, t0, b);
-            tma_load_4d(sm + OFF_RAW_K + x * 8192, &tm_k, &bar_load, 64 * x, h, t0, b);
-            tma_load_4d(sm + OFF_RAW_G + x * 8192, &tm_g, &bar_load, 64 * x, h, t0, b);
-            tma_load_4d(sm + OFF_RAW_V + x * 8192, &tm_v, &bar_load, 64 * x, h, t0, b);
+            tma_load_4d(sm + OFF_RAW_Q + x * 8192, &tm_q, &bar_qkg, 64 * x, h, chunk * kC, b);
+            tma_load_4d(sm + OFF_RAW_K + x * 8192, &tm_k, &bar_qkg, 64 * x, h, chunk * kC, b);
+            tma_load_4d(sm + OFF_RAW_G + x * 8192, &tm_g, &bar_qkg, 64 * x, h, chunk * kC, b);
         }
     };
-    int pending_chunk = -1;  // chunk whose TMA loads are in flight (meaningful in thread 0)
-    if (tid == 0 && nchunks > 0) {
-        issue_loads(0);
-        pending_chunk = 0;
-    }
-
-    // ---- initial state: fp32 into TMEM (TM_S), bf16 copy into the MN-major S tile ----
-    {
-        const int i = 32 * quarter + lane;  // state row (dk index) = TMEM lane
-        for (int cb = 0; cb < 64; cb += 16) {
-            const int c0 = 64 * colhalf + cb;
-            float r[16];
-            if (p.S0) {
-                const float4* src = reinterpret_cast<const float4*>(p.S0 + ((size_t)bh * kD + i) * kD + c0);
+    auto load_v = [&](int chunk) {
+        mbar_arrive_expect_tx(&bar_v, 16384u);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float4 x = src[j];
-                    r[4 * j] = x.x; r[4 * j + 1] = x.y; r[4 * j + 2] = x.z; r[4 * j + 3] = x.w;
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) r[j] = 0.f;
-            }
-            tmem_st16(tlane + TM_S + c0, r);
-#pragma unroll
-            for (int j = 0; j < 16; j += 8) {
-                uint4 pk;
-                pk.x = pack_bf16x2(r[j], r[j + 1]); pk.y = pack_bf16x2(r[j + 2], r[j + 3]);
-                pk.z = pack_bf16x2(r[j + 4], r[j + 5]); pk.w = pack_bf16x2(r[j + 6], r[j + 7]);
-                *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_offset(i, c0 + j, 16384)) = pk;
-            }
-        }
-        tmem_wait_st();
-    }
-    fence_proxy_async_smem();
-    tc_fence_before_sync();
-    __syncthreads();
+        for (int x = 0; x < 2; ++x) tma_load_4d(sm + OFF_V + x * 8192, &tm_v, &bar_v, 64 * x, h, chunk * kC, b);
+    };
 
     bool ok = true;
-    for (int chunk = 0; chunk < nchunks; ++chunk) {
-        const uint32_t par = chunk & 1;
-        const int t0 = chunk * kC;
-        const int nvalid = min(kC, T - t0);
-
-        if (tid < kC) {
-            const int t = t0 + tid;
-            s_beta[tid] = (t < T) ? __bfloat162float(p.beta[((size_t)b * T + t) * p.H + h]) : 0.f;
-        }
-        // Lower-triangular ones L[r][j] = (j <= r), bf16, K-major, 64 rows: the in-chunk cumulative
-        // sum of g as a tensor-core product (Gam = L g).  Rewritten every chunk because its home in
-        // the operand region is reused later in the chunk.
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int idx = tid + kThreads * e;  // 512 chunks of 8 elements
-            const int r = idx >> 3, j0 = (idx & 7) * 8;
-            uint4 pk;
-            uint32_t w[4];
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const uint32_t lo = (j0 + 2 * m <= r) ? 0x3F80u : 0u;
-                const uint32_t hi = (j0 + 2 * m + 1 <= r) ? 0x3F80u : 0u;
-                w[m] = lo | (hi << 16);
-            }
-            pk.x = w[0]; pk.y = w[1]; pk.z = w[2]; pk.w = w[3];
-            *reinterpret_cast<uint4*>(sm + OFF_L + sw128_offset(r, j0, 8192)) = pk;
-        }
-        fence_proxy_async_smem();
-        ok = mbar_wait(&bar_load, par, kTimeoutNs);
-        if (ok) pending_chunk = -1;
-        ok = __syncthreads_and(ok) != 0;
-        if (!ok) break;
-        if (tid == 0) {
-            tc_fence_after_sync();
-            // Gam for channels 0..63 into lanes 0..63 (rows 64..127 of A read other smem),
-            // channels 64..127 into lanes 64..127 (rows 0..63 of A read other smem)
-            issue_mma<4, false, 0, true, 8192>(tbase + TM_U, sb + OFF_L, sb + OFF_RAW_G, ID_G, false);
-            issue_mma<4, false, 0, true, 8192>(tbase + TM_U + 64, sb + OFF_L - 8192, sb + OFF_RAW_G + 8192, ID_G, false);
-            mma_commit(&bar_g);
-        }
-
-        // ================= step 2: decay factors and the bf16 operand tiles =================
-        // thread = one token row r and 32 channels c0..c0+31 (its TMEM lane holds Gam[r][c0..])
+    if (is_prep) {
+        // ====================================================================== prep group
+        const int ptid = tid;                               // 0..255
+        int pending = -1;                                   // chunk whose q,k,g loads are in flight
+        if (ptid == 0) { load_qkg(0); pending = 0; }
+        float* AF = reinterpret_cast<float*>(sm + OFF_AF);
+        float* XF = reinterpret_cast<float*>(sm + OFF_X);
+        float* XT = reinterpret_cast<float*>(sm + OFF_XT);
+        // token row / channel range of this thread in the element-wise step
         const int tr = 32 * (quarter & 1) + lane;            // token
         const int hf = quarter & 1;                          // 32-token block of the token
         const int jr = lane;                                 // row inside the block
-        const int c0 = 64 * (quarter >> 1) + 32 * colhalf;   // first channel
-        float* refs = reinterpret_cast<float*>(sm + OFF_CONST);          // [4][128] Gam rows 16,31,48,63
-        float* cst = refs + 4 * kD;                                       // per-channel constants
-        // cst layout: [hf][k][128] with k = 0: Gam_m*log2e, 1: e^{Gam_m}, 2: e^{Gam_63-Gam_m}, 3: c_off
-        uint32_t kb[16];  // Kb of this token row, bf16x2, stored once MMA1/2 have finished reading B1
-        {
+        const int c0 = 64 * (quarter >> 1) + 32 * colhalf;   // first of 32 channels
+        for (int chunk = 0; chunk < nchunks; ++chunk) {
+            const uint32_t par = chunk & 1, ppar = par ^ 1u;
+            const int t0 = chunk * kC;
+            // ---- P1: beta, L tile, Gam = L g on the tensor core
+            if (ptid < kC) {
+                const int t = t0 + ptid;
+                s_beta[ptid] = (t < T) ? __bfloat162float(p.beta[((size_t)b * T + t) * p.H + h]) : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int idx = ptid + kPrepThreads * e;  // 512 chunks of 8 elements
+                const int r = idx >> 3, j0 = (idx & 7) * 8;
+                uint32_t w[4];
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    w[m] = ((j0 + 2 * m <= r) ? 0x3F80u : 0u) | ((j0 + 2 * m + 1 <= r) ? 0x3F800000u : 0u);
+                *reinterpret_cast<uint4*>(sm + OFF_L + sw128_offset(r, j0, 8192)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            fence_proxy_async_smem();
+            if (ptid == 0) {
+                ok = mbar_wait(&bar_qkg, par, kTimeoutNs);
+                if (ok) pending = -1;
+            }
+            ok = named_bar_and(kBarPrep, kPrepThreads, ok);
+            if (!ok) break;
+            if (ptid == 0) {
+                tc_fence_after_sync();
+                // channels 0..63 into lanes 0..63 (A rows 64..127 read other smem),
+                // channels 64..127 into lanes 64..127 (A rows 0..63 read other smem)
+                issue_mma<4, false, 0, true, 8192>(tbase + TM_P, sb + OFF_L, sb + OFF_RAW_G, ID_G, false);
+                issue_mma<4, false, 0, true, 8192>(tbase + TM_P + 64, sb + OFF_L - 8192, sb + OFF_RAW_G + 8192,
+                                                   ID_G, false);
+                mma_commit(&bar_g);
+            }
+            // ---- P2: Gam rows and per-channel constants
             ok = mbar_wait(&bar_g, par, kTimeoutNs);
             tc_fence_after_sync();
             float G[32];
-            tmem_ld16(tlane + TM_U + c0, G);          // lanes 64.. hold channels 64.. (second MMA)
-            tmem_ld16(tlane + TM_U + c0 + 16, G + 16);
+            tmem_ld16(tlane + TM_P + c0, G);
+            tmem_ld16(tlane + TM_P + c0 + 16, G + 16);
             tmem_wait_ld();
-            const int refk = (lane == 16) ? 0 : (lane == 31) ? 1 : -1;
-            if (refk >= 0) {
-                float* dst = refs + (2 * hf + refk) * kD + c0;
+            if (lane == 16 || lane == 31) {
+                float* dst = &s_refs[2 * hf + (lane == 31)][c0];
 #pragma unroll
                 for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(G[e], G[e + 1], G[e + 2], G[e + 3]);
             }
-            ok = __syncthreads_and(ok) != 0;
+            ok = named_bar_and(kBarPrep, kPrepThreads, ok);
             if (!ok) break;
-            if (tid < kD) {
-                const float g16 = refs[tid], g31 = refs[kD + tid], g48 = refs[2 * kD + tid], g63 = refs[3 * kD + tid];
-                cst[0 * kD + tid] = g16 * kLog2e;
-                cst[1 * kD + tid] = expf(g16);
-                cst[2 * kD + tid] = expf(g63 - g16);
-                cst[3 * kD + tid] = expf(g31 - g16);
-                cst[4 * kD + tid] = g48 * kLog2e;
-                cst[5 * kD + tid] = expf(g48);
-                cst[6 * kD + tid] = expf(g63 - g48);
-                cst[7 * kD + tid] = expf(g48 - g31);
-                s_gammaC[tid] = expf(g63);
+            if (ptid < kD) {
+                const float g16 = s_refs[0][ptid], g48 = s_refs[2][ptid], g63 = s_refs[3][ptid];
+                s_cst[0][0][ptid] = g16 * kLog2e;
+                s_cst[0][1][ptid] = expf(g16);
+                s_cst[0][2][ptid] = expf(g63 - g16);
+                s_cst[0][3][ptid] = expf(g48 - g16);    // block-0 columns: reference 16 -> 48
+                s_cst[1][0][ptid] = g48 * kLog2e;
+                s_cst[1][1][ptid] = expf(g48);
+                s_cst[1][2][ptid] = expf(g63 - g48);
+                s_cst[1][3][ptid] = 0.f;
+                s_gamma[par][ptid] = expf(g63);
             }
-            __syncthreads();
-            const float* ch = cst + 4 * kD * hf;
+            // ---- P3: operand tiles (KQ may be rewritten once MMA3 of the previous chunk is done)
+            if (chunk > 0) ok = mbar_wait(&bar_c, ppar, kTimeoutNs);
+            ok = named_bar_and(kBarPrep, kPrepThreads, ok);
+            if (!ok) break;
+            uint32_t kb[16];  // Kb of this token row, written once the previous chunk released the tile
 #pragma unroll
             for (int g8 = 0; g8 < 4; ++g8) {
                 const int cc = c0 + 8 * g8;
@@ -343,17 +325,20 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const uint4 qraw = *reinterpret_cast<const uint4*>(sm + OFF_RAW_Q + roff);
                 const uint4 kraw = *reinterpret_cast<const uint4*>(sm + OFF_RAW_K + roff);
                 float gmL[8], cm[8], ce[8], co[8];
-                *reinterpret_cast<float4*>(gmL) = *reinterpret_cast<const float4*>(ch + 0 * kD + cc);
-                *reinterpret_cast<float4*>(gmL + 4) = *reinterpret_cast<const float4*>(ch + 0 * kD + cc + 4);
-                *reinterpret_cast<float4*>(cm) = *reinterpret_cast<const float4*>(ch + 1 * kD + cc);
-                *reinterpret_cast<float4*>(cm + 4) = *reinterpret_cast<const float4*>(ch + 1 * kD + cc + 4);
-                *reinterpret_cast<float4*>(ce) = *reinterpret_cast<const float4*>(ch + 2 * kD + cc);
-                *reinterpret_cast<float4*>(ce + 4) = *reinterpret_cast<const float4*>(ch + 2 * kD + cc + 4);
-                *reinterpret_cast<float4*>(co) = *reinterpret_cast<const float4*>(ch + 3 * kD + cc);
-                *reinterpret_cast<float4*>(co + 4) = *reinterpret_cast<const float4*>(ch + 3 * kD + cc + 4);
+#pragma unroll
+                for (int u = 0; u < 8; u += 4) {
+                    const float4 x0 = *reinterpret_cast<const float4*>(&s_cst[hf][0][cc + u]);
+                    const float4 x1 = *reinterpret_cast<const float4*>(&s_cst[hf][1][cc + u]);
+                    const float4 x2 = *reinterpret_cast<const float4*>(&s_cst[hf][2][cc + u]);
+                    const float4 x3 = *reinterpret_cast<const float4*>(&s_cst[hf][3][cc + u]);
+                    gmL[u] = x0.x; gmL[u + 1] = x0.y; gmL[u + 2] = x0.z; gmL[u + 3] = x0.w;
+                    cm[u] = x1.x; cm[u + 1] = x1.y; cm[u + 2] = x1.z; cm[u + 3] = x1.w;
+                    ce[u] = x2.x; ce[u + 1] = x2.y; ce[u + 2] = x2.z; ce[u + 3] = x2.w;
+                    co[u] = x3.x; co[u + 1] = x3.y; co[u + 2] = x3.z; co[u + 3] = x3.w;
+                }
                 const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qraw);
                 const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kraw);
-                uint32_t a1q[4], a1k[4], b1[4], kqk[4], kqq[4], x1[4], x2[4];
+                uint32_t a1q[4], a1k[4], b1[4], kqk[4], kqq[4], bx[4];
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
                     const float2 qf = __bfloat1622float2(q2[m]);
@@ -371,178 +356,163 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     a1q[m] = pack_bf16x2(qE0, qE1);
                     a1k[m] = pack_bf16x2(kE0, kE1);
                     b1[m] = pack_bf16x2(kI0, kI1);
-                    kqk[m] = pack_bf16x2(kE0 * cm[2 * m], kE1 * cm[2 * m + 1]);
                     kqq[m] = pack_bf16x2(qE0 * cm[2 * m], qE1 * cm[2 * m + 1]);
+                    kqk[m] = pack_bf16x2(kE0 * cm[2 * m], kE1 * cm[2 * m + 1]);
                     kb[4 * g8 + m] = pack_bf16x2(kI0 * ce[2 * m], kI1 * ce[2 * m + 1]);
-                    if (hf) {
-                        x1[m] = pack_bf16x2(qE0 * co[2 * m], qE1 * co[2 * m + 1]);
-                        x2[m] = pack_bf16x2(kE0 * co[2 * m], kE1 * co[2 * m + 1]);
-                    } else {
-                        x1[m] = pack_bf16x2(kI0 * co[2 * m], kI1 * co[2 * m + 1]);
-                    }
+                    bx[m] = pack_bf16x2(kI0 * co[2 * m], kI1 * co[2 * m + 1]);
                 }
-                // MMA1 operands: rows [Qt0; Kt0; Qt1; Kt1] and [Kh0; Kh1] against the block middles
+                // MMA1 operands: A rows [Qt0;Kt0;Qt1;Kt1], B rows [Kh0(16);Kh1(48);Kh0(48)]
                 *reinterpret_cast<uint4*>(sm + OFF_A1 + sw128_offset(64 * hf + jr, cc, 16384)) = make_uint4(a1q[0], a1q[1], a1q[2], a1q[3]);
                 *reinterpret_cast<uint4*>(sm + OFF_A1 + sw128_offset(64 * hf + 32 + jr, cc, 16384)) = make_uint4(a1k[0], a1k[1], a1k[2], a1k[3]);
-                *reinterpret_cast<uint4*>(sm + OFF_B1 + sw128_offset(tr, cc, 8192)) = make_uint4(b1[0], b1[1], b1[2], b1[3]);
-                // MMA3 operand [Kt; Qt] against the chunk start
-                *reinterpret_cast<uint4*>(sm + OFF_KQ + sw128_offset(tr, cc, 16384)) = make_uint4(kqk[0], kqk[1], kqk[2], kqk[3]);
-                *reinterpret_cast<uint4*>(sm + OFF_KQ + sw128_offset(64 + tr, cc, 16384)) = make_uint4(kqq[0], kqq[1], kqq[2], kqq[3]);
-                if (hf) {  // MMA2 rows: block 1 against token 31, stored as rows 64..127 of a virtual tile
-                    *reinterpret_cast<uint4*>(sm + OFF_A2 + sw128_offset(jr, cc, 8192)) = make_uint4(x1[0], x1[1], x1[2], x1[3]);
-                    *reinterpret_cast<uint4*>(sm + OFF_A2 + sw128_offset(32 + jr, cc, 8192)) = make_uint4(x2[0], x2[1], x2[2], x2[3]);
-                } else {   // MMA2 columns: block 0 against token 31
-                    *reinterpret_cast<uint4*>(sm + OFF_B2 + sw128_offset(jr, cc, 4096)) = make_uint4(x1[0], x1[1], x1[2], x1[3]);
-                }
+                *reinterpret_cast<uint4*>(sm + OFF_BB + sw128_offset(tr, cc, 12288)) = make_uint4(b1[0], b1[1], b1[2], b1[3]);
+                if (hf == 0)
+                    *reinterpret_cast<uint4*>(sm + OFF_BB + sw128_offset(64 + jr, cc, 12288)) = make_uint4(bx[0], bx[1], bx[2], bx[3]);
+                // MMA3 operand: the same row order against the chunk start
+                *reinterpret_cast<uint4*>(sm + OFF_KQ + sw128_offset(64 * hf + jr, cc, 16384)) = make_uint4(kqq[0], kqq[1], kqq[2], kqq[3]);
+                *reinterpret_cast<uint4*>(sm + OFF_KQ + sw128_offset(64 * hf + 32 + jr, cc, 16384)) = make_uint4(kqk[0], kqk[1], kqk[2], kqk[3]);
             }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
-
-        if (tid == 0) {
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            named_bar_sync(kBarPrep, kPrepThreads);
+            if (ptid == 0) {
+                tc_fence_after_sync();
+                mbar_arrive(&bar_kq);  // KQ of this chunk is ready for MMA3
+                issue_mma<8, false, 16384, false, 12288>(tbase + TM_P, sb + OFF_A1, sb + OFF_BB, ID_MMA1, false);
+                mma_commit(&bar_ap);
+                // raw q,k,g are consumed (Gam was read before the barrier): prefetch the next chunk
+                if (chunk + 1 < nchunks) { load_qkg(chunk + 1); pending = chunk + 1; }
+            }
+            // ---- P4: P and A from TMEM, Kb tile, triangular solve, T tile
+            ok = mbar_wait(&bar_ap, par, kTimeoutNs);
+            if (ok && chunk > 0) ok = mbar_wait(&bar_os, ppar, kTimeoutNs);  // T, P, Kb released
             tc_fence_after_sync();
-            issue_mma<8, false, 16384, false, 8192>(tbase + TM_AP, sb + OFF_A1, sb + OFF_B1, ID_MMA1, false);
-            issue_mma<8, false, 8192, false, 4096>(tbase + TM_AP + 64, sb + OFF_A2 - 8192, sb + OFF_B2, ID_MMA2, false);
-            mma_commit(&bar_ap);
-            issue_mma<8, false, 16384, true, 16384>(tbase + TM_C, sb + OFF_KQ, sb + OFF_SB, ID_KxMN, false);
-            mma_commit(&bar_c);
-        }
-
-        // ================= step 3: P and A from TMEM; Kb tile; diagonal blocks of (I+A)^-1 =========
-        ok = mbar_wait(&bar_ap, par, kTimeoutNs);
-        tc_fence_after_sync();
-        ok = __syncthreads_and(ok) != 0;
-        if (!ok) break;
-        float* AF = reinterpret_cast<float*>(sm + OFF_AF);   // A, fp32, row stride kLd
-        float* XF = reinterpret_cast<float*>(sm + OFF_X);    // X = (I+A)^-1, row-major
-        float* XT = reinterpret_cast<float*>(sm + OFF_XT);   // X transposed
+            ok = named_bar_and(kBarPrep, kPrepThreads, ok);
+            if (!ok) break;
 #pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8)
-            *reinterpret_cast<uint4*>(sm + OFF_KBAR + sw128_offset(tr, c0 + 8 * g8, 8192)) =
-                make_uint4(kb[4 * g8], kb[4 * g8 + 1], kb[4 * g8 + 2], kb[4 * g8 + 3]);
-        if (warp < 4) {
-            // lane L of TM_AP: L < 32: Qt0 row r = L; L < 64: Kt0 row r = L - 32;
-            //                  L < 96: Qt1 row r = L - 32; else Kt1 row r = L - 64.
-            const int L = 32 * warp + lane;
-            const bool is_q = (warp == 0) || (warp == 2);
-            const int r = (L < 64) ? (L & 31) : 32 + (L & 31);
-            float row[64];
-            if (warp < 2) {
+            for (int g8 = 0; g8 < 4; ++g8)
+                *reinterpret_cast<uint4*>(sm + OFF_KBAR + sw128_offset(tr, c0 + 8 * g8, 8192)) =
+                    make_uint4(kb[4 * g8], kb[4 * g8 + 1], kb[4 * g8 + 2], kb[4 * g8 + 3]);
+            {
+                // TMEM lane L of MMA1: quarter 0 Qt0 rows, 1 Kt0 rows, 2 Qt1 rows, 3 Kt1 rows.
+                // Columns of a row r: j < 32 from cols 0..31 (block 0) or 64..95 (block 1 rows);
+                // j >= 32 zero (block 0) or cols 32..63 (block 1).  colhalf picks j < 32 / j >= 32.
+                const bool is_q = (quarter & 1) == 0;
+                const int r = 32 * (quarter >> 1) + lane;
+                const int jb = 32 * colhalf;
+                float row[32];
+                if (quarter < 2) {
+                    if (colhalf == 0) {
+                        tmem_ld16(tlane + TM_P, row);
+                        tmem_ld16(tlane + TM_P + 16, row + 16);
+                        tmem_wait_ld();
+                    } else {
 #pragma unroll
-                for (int cb = 0; cb < 32; cb += 16) tmem_ld16(tlane + TM_AP + cb, row + cb);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 32; j < 64; ++j) row[j] = 0.f;
-            } else {
-                // MMA2 columns 0..31: off-diagonal block (j = 0..31); MMA1 columns 32..63: block 1 (j = 32..63)
-#pragma unroll
-                for (int cb = 0; cb < 32; cb += 16) tmem_ld16(tlane + TM_AP + 64 + cb, row + cb);
-#pragma unroll
-                for (int cb = 0; cb < 32; cb += 16) tmem_ld16(tlane + TM_AP + 32 + cb, row + 32 + cb);
-                tmem_wait_ld();
-            }
-            if (is_q) {
-                // P row r: lower triangle including the diagonal, bf16, rows 64.. of the P tile
-#pragma unroll
-                for (int j = 0; j < 64; j += 8) {
-                    float v8[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) v8[e] = (j + e <= r) ? row[j + e] : 0.f;
-                    *reinterpret_cast<uint4*>(sm + OFF_PV + 8192 + sw128_offset(r, j, 8192)) =
-                        make_uint4(pack_bf16x2(v8[0], v8[1]), pack_bf16x2(v8[2], v8[3]),
-                                   pack_bf16x2(v8[4], v8[5]), pack_bf16x2(v8[6], v8[7]));
-                }
-            } else {
-                // A row r: strictly lower, scaled by beta_r (select first: masked entries may be inf)
-                const float br = s_beta[r];
-#pragma unroll
-                for (int j = 0; j < 64; ++j) row[j] = (j < r) ? br * row[j] : 0.f;
-#pragma unroll
-                for (int j = 0; j < 64; j += 4)
-                    *reinterpret_cast<float4*>(AF + r * kLd + j) = make_float4(row[j], row[j + 1], row[j + 2], row[j + 3]);
-                // diagonal 16x16 block of X = (I + A)^-1 by forward substitution across the
-                // 16 lanes that own its rows (two blocks per warp, one per half-warp)
-                const int s16 = r & 15, blk = r >> 4, base = lane & 16;
-                float dg[16];
-                if (warp == 1) {
-#pragma unroll
-                    for (int t = 0; t < 16; ++t) dg[t] = (lane < 16) ? row[t] : row[16 + t];
+                        for (int j = 0; j < 32; ++j) row[j] = 0.f;
+                    }
                 } else {
-#pragma unroll
-                    for (int t = 0; t < 16; ++t) dg[t] = (lane < 16) ? row[32 + t] : row[48 + t];
+                    const uint32_t col = colhalf == 0 ? 64u : 32u;
+                    tmem_ld16(tlane + TM_P + col, row);
+                    tmem_ld16(tlane + TM_P + col + 16, row + 16);
+                    tmem_wait_ld();
                 }
+                if (is_q) {
+                    // P row r: lower triangle including the diagonal
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) {
+                        float v8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v8[e] = (jb + j + e <= r) ? row[j + e] : 0.f;
+                        *reinterpret_cast<uint4*>(sm + OFF_P + sw128_offset(tp_row(r), jb + j, 8192)) = pack8(v8);
+                    }
+                } else {
+                    // A row r: strictly lower, scaled by beta_r (select first: masked entries may be inf)
+                    const float br = s_beta[r];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        float4 w4;
+                        w4.x = (jb + j + 0 < r) ? br * row[j + 0] : 0.f;
+                        w4.y = (jb + j + 1 < r) ? br * row[j + 1] : 0.f;
+                        w4.z = (jb + j + 2 < r) ? br * row[j + 2] : 0.f;
+                        w4.w = (jb + j + 3 < r) ? br * row[j + 3] : 0.f;
+                        *reinterpret_cast<float4*>(AF + r * kLd + jb + j) = w4;
+                    }
+                }
+            }
+            tc_fence_before_sync();  // the next chunk's Gam product reuses these TMEM columns
+            named_bar_sync(kBarPrep, kPrepThreads);
+            // diagonal 16x16 blocks of X = (I + A)^-1 by forward substitution, one lane per column:
+            // x_r = e_c[r] - sum_{l<r} A[r][l] x_l (the strictly upper entries of A are stored as 0)
+            if (warp < 2) {
+                const int blk = 2 * warp + (lane >> 4), c = lane & 15, o0 = 16 * blk;
                 float x[16];
 #pragma unroll
-                for (int c = 0; c < 16; ++c) x[c] = (c == s16) ? 1.f : 0.f;
+                for (int r = 0; r < 16; ++r) {
+                    const float* ar = AF + (o0 + r) * kLd + o0;
+                    float s0 = (r == c) ? 1.f : 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-                for (int t = 0; t < 15; ++t) {
-                    float xt[16];
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) xt[c] = __shfl_sync(0xffffffffu, x[c], base + t);
-                    if (s16 > t) {
-#pragma unroll
-                        for (int c = 0; c < 16; ++c) x[c] = fmaf(-dg[t], xt[c], x[c]);
+                    for (int l = 0; l < (r & ~3); l += 4) {
+                        const float4 a4 = *reinterpret_cast<const float4*>(ar + l);
+                        s0 = fmaf(-a4.x, x[l], s0); s1 = fmaf(-a4.y, x[l + 1], s1);
+                        s2 = fmaf(-a4.z, x[l + 2], s2); s3 = fmaf(-a4.w, x[l + 3], s3);
                     }
+#pragma unroll
+                    for (int l = (r & ~3); l < r; ++l) s0 = fmaf(-ar[l], x[l], s0);
+                    x[r] = (s0 + s1) + (s2 + s3);
                 }
 #pragma unroll
-                for (int c = 0; c < 16; c += 4)
-                    *reinterpret_cast<float4*>(XF + r * kLd + 16 * blk + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
+                for (int r = 0; r < 16; ++r) XF[(o0 + r) * kLd + o0 + c] = x[r];
 #pragma unroll
-                for (int c = 0; c < 16; ++c) XT[(16 * blk + c) * kLd + r] = x[c];
+                for (int r = 0; r < 16; r += 4)
+                    *reinterpret_cast<float4*>(XT + (o0 + c) * kLd + o0 + r) = make_float4(x[r], x[r + 1], x[r + 2], x[r + 3]);
             }
-        }
-        __syncthreads();
-
-        // ================= step 4: off-diagonal blocks of X, then T = X Diag(beta) ================
-        // X_RJ = -X_RR sum_{L=J}^{R-1} A_RL X_LJ, by block distance d = R - J (16x16 blocks), on
-        // warp-level bf16 tensor-core tiles with fp32 accumulation (the chunk model shows bf16
-        // operands here leave the output error unchanged).  Warp 2*qb + nt computes the 8 output
-        // columns nt of block qb of the level.
-        {
-            const int g4 = lane >> 2, t4 = lane & 3;
-            float* WS = reinterpret_cast<float*>(sm + OFF_WS) + warp * 8 * kLdS;  // this warp's W^T (8 x 16)
+            named_bar_sync(kBarPrep, kPrepThreads);
+            // X_RJ = -X_RR sum_{L=J}^{R-1} A_RL X_LJ by block distance d = R - J on warp-level bf16
+            // tensor-core tiles, fp32 accumulation (bf16 operands here leave the output error
+            // unchanged in the chunk model).  Warp 2*qb + nt: 8 output columns nt of block qb.
+            {
+                const int g4 = lane >> 2, t4 = lane & 3;
+                float* WS = reinterpret_cast<float*>(sm + OFF_WS) + warp * 8 * kLdS;
 #pragma unroll
-            for (int d = 1; d < 4; ++d) {
-                if (warp < 2 * (4 - d)) {
-                    const int qb = warp >> 1, nt = warp & 1;
-                    const int R = qb + d, J = qb;
-                    float w[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int d = 1; d < 4; ++d) {
+                    if (warp < 2 * (4 - d)) {
+                        const int qb = warp >> 1, nt = warp & 1;
+                        const int R = qb + d, J = qb;
+                        float w[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int Lb = 0; Lb < 3; ++Lb) {
-                        if (Lb < d) {
-                            const int L = J + Lb;
-                            uint32_t af[4], bf[2];
-                            load_a_frag(AF + (16 * R) * kLd + 16 * L, kLd, g4, t4, af);
-                            load_b_frag(XT + (16 * J + 8 * nt) * kLd + 16 * L, kLd, g4, t4, bf);
-                            mma_16816(w, af, bf);
+                        for (int Lb = 0; Lb < 3; ++Lb) {
+                            if (Lb < d) {
+                                const int L = J + Lb;
+                                uint32_t af[4], bf[2];
+                                load_a_frag(AF + (16 * R) * kLd + 16 * L, kLd, g4, t4, af);
+                                load_b_frag(XT + (16 * J + 8 * nt) * kLd + 16 * L, kLd, g4, t4, bf);
+                                mma_16816(w, af, bf);
+                            }
                         }
+                        WS[(2 * t4) * kLdS + g4] = w[0];
+                        WS[(2 * t4 + 1) * kLdS + g4] = w[1];
+                        WS[(2 * t4) * kLdS + g4 + 8] = w[2];
+                        WS[(2 * t4 + 1) * kLdS + g4 + 8] = w[3];
+                        __syncwarp();
+                        uint32_t af[4], bf[2];
+                        load_a_frag(XF + (16 * R) * kLd + 16 * R, kLd, g4, t4, af);
+                        load_b_frag(WS, kLdS, g4, t4, bf);
+                        float x[4] = {0.f, 0.f, 0.f, 0.f};
+                        mma_16816(x, af, bf);
+                        const int col = 16 * J + 8 * nt + 2 * t4;
+                        *reinterpret_cast<float2*>(XF + (16 * R + g4) * kLd + col) = make_float2(-x[0], -x[1]);
+                        *reinterpret_cast<float2*>(XF + (16 * R + g4 + 8) * kLd + col) = make_float2(-x[2], -x[3]);
+                        XT[col * kLd + 16 * R + g4] = -x[0];
+                        XT[(col + 1) * kLd + 16 * R + g4] = -x[1];
+                        XT[col * kLd + 16 * R + g4 + 8] = -x[2];
+                        XT[(col + 1) * kLd + 16 * R + g4 + 8] = -x[3];
                     }
-                    // W (16 x 8, this warp's columns) -> transposed scratch, read back as the B fragment
-                    WS[(2 * t4) * kLdS + g4] = w[0];
-                    WS[(2 * t4 + 1) * kLdS + g4] = w[1];
-                    WS[(2 * t4) * kLdS + g4 + 8] = w[2];
-                    WS[(2 * t4 + 1) * kLdS + g4 + 8] = w[3];
-                    __syncwarp();
-                    uint32_t af[4], bf[2];
-                    load_a_frag(XF + (16 * R) * kLd + 16 * R, kLd, g4, t4, af);
-                    load_b_frag(WS, kLdS, g4, t4, bf);
-                    float x[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_16816(x, af, bf);
-                    const int col = 16 * J + 8 * nt + 2 * t4;
-                    *reinterpret_cast<float2*>(XF + (16 * R + g4) * kLd + col) = make_float2(-x[0], -x[1]);
-                    *reinterpret_cast<float2*>(XF + (16 * R + g4 + 8) * kLd + col) = make_float2(-x[2], -x[3]);
-                    XT[col * kLd + 16 * R + g4] = -x[0];
-                    XT[(col + 1) * kLd + 16 * R + g4] = -x[1];
-                    XT[col * kLd + 16 * R + g4 + 8] = -x[2];
-                    XT[(col + 1) * kLd + 16 * R + g4 + 8] = -x[3];
+                    named_bar_sync(kBarPrep, kPrepThreads);
                 }
-                __syncthreads();
             }
-            // T = X Diag(beta) -> bf16 K-major tile rows 0..63 (K = 64 tokens); upper blocks are 0
+            // T = X Diag(beta), bf16, K-major (K = 64 tokens); strictly upper blocks are 0
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const int idx = tid + kThreads * e;  // 512 chunks of 8
+                const int idx = ptid + kPrepThreads * e;  // 512 chunks of 8
                 const int r = idx >> 3, j = (idx & 7) * 8;
                 uint4 pk = make_uint4(0u, 0u, 0u, 0u);
                 if ((j >> 4) <= (r >> 4)) {
@@ -553,155 +523,185 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     pk.z = pack_bf16x2(xb.x * s_beta[j + 4], xb.y * s_beta[j + 5]);
                     pk.w = pack_bf16x2(xb.z * s_beta[j + 6], xb.w * s_beta[j + 7]);
                 }
-                *reinterpret_cast<uint4*>(sm + OFF_T + sw128_offset(r, j, 8192)) = pk;
+                *reinterpret_cast<uint4*>(sm + OFF_T + sw128_offset(tp_row(r), j, 8192)) = pk;
             }
+            fence_proxy_async_smem();
+            named_bar_sync(kBarPrep, kPrepThreads);
+            if (ptid == 0) mbar_arrive(&bar_tpk);  // T, P, Kb and gamma of this chunk are ready
         }
-
-        // ================= step 5: Y = V - Kt S  (TMEM lanes 0..63 of TM_C) =================
-        ok = mbar_wait(&bar_c, par, kTimeoutNs);
-        tc_fence_after_sync();
-        ok = __syncthreads_and(ok) != 0;
-        if (!ok) break;
-        if (quarter < 2) {
-            const int r = 32 * quarter + lane;
-            float ks[64];
-#pragma unroll
-            for (int cb = 0; cb < 64; cb += 16) tmem_ld16(tlane + TM_C + 64 * colhalf + cb, ks + cb);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 64; j += 8) {
-                const uint32_t off = sw128_offset(r, 64 * colhalf + j, 8192);
-                const uint4 vv = *reinterpret_cast<const uint4*>(sm + OFF_RAW_V + off);
-                const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vv);
-                uint4 pk;
-                float2 f;
-                f = __bfloat1622float2(v2[0]); pk.x = pack_bf16x2(f.x - ks[j + 0], f.y - ks[j + 1]);
-                f = __bfloat1622float2(v2[1]); pk.y = pack_bf16x2(f.x - ks[j + 2], f.y - ks[j + 3]);
-                f = __bfloat1622float2(v2[2]); pk.z = pack_bf16x2(f.x - ks[j + 4], f.y - ks[j + 5]);
-                f = __bfloat1622float2(v2[3]); pk.w = pack_bf16x2(f.x - ks[j + 6], f.y - ks[j + 7]);
-                *reinterpret_cast<uint4*>(sm + OFF_YU + off) = pk;
-            }
+        if (!ok && ptid == 0) report_status(p.status, KDA_ERR_TIMEOUT);
+        // drain: no MMA or TMA issued by this group may still be in flight
+        if (ptid == 0) {
+            mma_commit(&bar_drain_p);
+            if (!mbar_wait(&bar_drain_p, 0, kTimeoutNs)) report_status(p.status, KDA_ERR_TIMEOUT);
+            if (pending >= 0) (void)mbar_wait(&bar_qkg, (uint32_t)(pending & 1), kTimeoutNs);
         }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after_sync();
-            // raw tiles are all consumed: prefetch the next chunk
-            if (chunk + 1 < nchunks) {
-                issue_loads(chunk + 1);
-                pending_chunk = chunk + 1;
-            }
-            issue_mma<4, false, 0, true, 8192>(tbase + TM_U, sb + OFF_T, sb + OFF_YU, ID_KxMN, false);
-            mma_commit(&bar_u);
-        }
-
-        // ================= step 7: decay the fp32 state in TMEM; U -> bf16 tile =================
-        {
-            float sv[64];
-#pragma unroll
-            for (int cb = 0; cb < 64; cb += 16) tmem_ld16(tlane + TM_S + 64 * colhalf + cb, sv + cb);
-            tmem_wait_ld();
-            const float gc = s_gammaC[32 * quarter + lane];
-#pragma unroll
-            for (int j = 0; j < 64; ++j) sv[j] *= gc;
-#pragma unroll
-            for (int cb = 0; cb < 64; cb += 16) tmem_st16(tlane + TM_S + 64 * colhalf + cb, sv + cb);
-            tmem_wait_st();
-        }
-        ok = mbar_wait(&bar_u, par, kTimeoutNs);
-        tc_fence_after_sync();
-        ok = __syncthreads_and(ok) != 0;
-        if (!ok) break;
-        if (quarter < 2) {
-            const int r = 32 * quarter + lane;
-            float u[64];
-#pragma unroll
-            for (int cb = 0; cb < 64; cb += 16) tmem_ld16(tlane + TM_U + 64 * colhalf + cb, u + cb);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 64; j += 8)
-                *reinterpret_cast<uint4*>(sm + OFF_YU + sw128_offset(r, 64 * colhalf + j, 8192)) =
-                    make_uint4(pack_bf16x2(u[j], u[j + 1]), pack_bf16x2(u[j + 2], u[j + 3]),
-                               pack_bf16x2(u[j + 4], u[j + 5]), pack_bf16x2(u[j + 6], u[j + 7]));
-        }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after_sync();
-            // O = Qt S + P U (onto lanes 64..127 of TM_C); S <- Diag(gamma_C) S + Kb^T U
-            issue_mma<4, false, 0, true, 8192>(tbase + TM_C, sb + OFF_PV, sb + OFF_YU, ID_KxMN, true);
-            issue_mma<4, true, 8192, true, 8192>(tbase + TM_S, sb + OFF_KBAR, sb + OFF_YU, ID_MNxMN, true);
-            mma_commit(&bar_os);
-        }
-
-        // ================= step 9: O -> global; S -> bf16 tile for the next chunk =================
-        ok = mbar_wait(&bar_os, par, kTimeoutNs);
-        tc_fence_after_sync();
-        ok = __syncthreads_and(ok) != 0;
-        if (!ok) break;
-        if (quarter >= 2) {
-            const int r = 32 * (quarter - 2) + lane;
-            // tcgen05.ld is warp-collective: every lane loads, only valid tokens are stored
-            float ov[64];
-#pragma unroll
-            for (int cb = 0; cb < 64; cb += 16) tmem_ld16(tlane + TM_C + 64 * colhalf + cb, ov + cb);
-            tmem_wait_ld();
-            if (r < nvalid) {
-                uint4* orow = reinterpret_cast<uint4*>(p.o + (((size_t)b * T + t0 + r) * p.H + h) * kD + 64 * colhalf);
-#pragma unroll
-                for (int j = 0; j < 64; j += 8)
-                    orow[j >> 3] = make_uint4(pack_bf16x2(ov[j], ov[j + 1]), pack_bf16x2(ov[j + 2], ov[j + 3]),
-                                              pack_bf16x2(ov[j + 4], ov[j + 5]), pack_bf16x2(ov[j + 6], ov[j + 7]));
-            }
-        }
+    } else {
+        // ====================================================================== serial group
+        const int stid = tid - kPrepThreads;                // 0..255
+        int pending = -1;                                   // chunk whose v load is in flight
+        // initial state: fp32 into TMEM, bf16 copy into the MN-major S tile
         {
             const int i = 32 * quarter + lane;
-            float sv[64];
+            const int cb0 = 64 * colhalf;
+            float r[64];
+            if (p.S0) {
+                const float4* src = reinterpret_cast<const float4*>(p.S0 + ((size_t)bh * kD + i) * kD + cb0);
 #pragma unroll
-            for (int cb = 0; cb < 64; cb += 16) tmem_ld16(tlane + TM_S + 64 * colhalf + cb, sv + cb);
-            tmem_wait_ld();
+                for (int j = 0; j < 16; ++j) {
+                    const float4 x = src[j];
+                    r[4 * j] = x.x; r[4 * j + 1] = x.y; r[4 * j + 2] = x.z; r[4 * j + 3] = x.w;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 64; ++j) r[j] = 0.f;
+            }
+#pragma unroll
+            for (int cb = 0; cb < 64; cb += 16) tmem_st16(tlane + TM_S + cb0 + cb, r + cb);
+            tmem_wait_st();
 #pragma unroll
             for (int j = 0; j < 64; j += 8)
-                *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_offset(i, 64 * colhalf + j, 16384)) =
-                    make_uint4(pack_bf16x2(sv[j], sv[j + 1]), pack_bf16x2(sv[j + 2], sv[j + 3]),
-                               pack_bf16x2(sv[j + 4], sv[j + 5]), pack_bf16x2(sv[j + 6], sv[j + 7]));
+                *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_offset(i, cb0 + j, 16384)) = pack8(r + j);
         }
+        if (stid == 0 && nchunks > 0) { load_v(0); pending = 0; }
         fence_proxy_async_smem();
         tc_fence_before_sync();
-        __syncthreads();
-    }
-
-    if (!ok && tid == 0) report_status(p.status, KDA_ERR_TIMEOUT);
-    // ---- drain: no tensor-core work or TMA may be in flight when the CTA exits ----
-    if (tid == 0) {
-        mma_commit(&bar_drain);
-        if (!mbar_wait(&bar_drain, 0, kTimeoutNs)) report_status(p.status, KDA_ERR_TIMEOUT);
-        if (pending_chunk >= 0) {
-            // a prefetch may still be landing: wait for it (bounded) before the smem is released
-            (void)mbar_wait(&bar_load, (uint32_t)(pending_chunk & 1), kTimeoutNs);
+        named_bar_sync(kBarSerial, kSerialThreads);
+        for (int chunk = 0; chunk < nchunks; ++chunk) {
+            const uint32_t par = chunk & 1;
+            const int t0 = chunk * kC;
+            const int nvalid = min(kC, T - t0);
+            // ---- S1: MMA3 = [Qt0;Kt0;Qt1;Kt1] S once the prep group has the KQ tile
+            if (stid == 0) {
+                ok = mbar_wait(&bar_kq, par, kTimeoutNs);
+                if (ok) {
+                    tc_fence_after_sync();
+                    issue_mma<8, false, 16384, true, 16384>(tbase + TM_C, sb + OFF_KQ, sb + OFF_SB, ID_KxMN, false);
+                    mma_commit(&bar_c);
+                }
+            }
+            // Y = V - Kt S (Kt rows sit in lanes 32-63 and 96-127), in place over v
+            if (ok) ok = mbar_wait(&bar_c, par, kTimeoutNs);
+            if (ok) ok = mbar_wait(&bar_v, par, kTimeoutNs);
+            tc_fence_after_sync();
+            ok = named_bar_and(kBarSerial, kSerialThreads, ok);
+            if (!ok) break;
+            if (stid == 0) pending = -1;
+            if (quarter & 1) {
+                const int tj = 32 * (quarter >> 1) + lane;
+                float ks[64];
+                tmem_ld64(tlane + TM_C + 64 * colhalf, ks);
+#pragma unroll
+                for (int j = 0; j < 64; j += 8) {
+                    const uint32_t off = sw128_offset(tj, 64 * colhalf + j, 8192);
+                    const uint4 vv = *reinterpret_cast<const uint4*>(sm + OFF_V + off);
+                    const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&vv);
+                    float y[8];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float2 f = __bfloat1622float2(v2[m]);
+                        y[2 * m] = f.x - ks[j + 2 * m];
+                        y[2 * m + 1] = f.y - ks[j + 2 * m + 1];
+                    }
+                    *reinterpret_cast<uint4*>(sm + OFF_V + off) = pack8(y);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            named_bar_sync(kBarSerial, kSerialThreads);
+            // ---- S2: MMA4 U = T Y once the prep group has T, P, Kb; decay the state meanwhile
+            if (stid == 0) {
+                ok = mbar_wait(&bar_tpk, par, kTimeoutNs);
+                if (ok) {
+                    tc_fence_after_sync();
+                    issue_mma<4, false, 0, true, 8192>(tbase + TM_U, sb + OFF_T, sb + OFF_V, ID_KxMN, false);
+                    mma_commit(&bar_u);
+                }
+            }
+            ok = named_bar_and(kBarSerial, kSerialThreads, ok);
+            if (!ok) break;
+            {
+                // S <- Diag(e^{Gam_63}) S in TMEM (gamma was published before T/P/Kb)
+                float sv[64];
+                tmem_ld64(tlane + TM_S + 64 * colhalf, sv);
+                const float gc = s_gamma[par][32 * quarter + lane];
+#pragma unroll
+                for (int j = 0; j < 64; ++j) sv[j] *= gc;
+#pragma unroll
+                for (int cb = 0; cb < 64; cb += 16) tmem_st16(tlane + TM_S + 64 * colhalf + cb, sv + cb);
+                tmem_wait_st();
+            }
+            ok = mbar_wait(&bar_u, par, kTimeoutNs);
+            tc_fence_after_sync();
+            ok = named_bar_and(kBarSerial, kSerialThreads, ok);
+            if (!ok) break;
+            // U (lanes 0-31 tokens 0-31, lanes 64-95 tokens 32-63) -> bf16, in place over Y
+            if ((quarter & 1) == 0) {
+                const int tj = 32 * (quarter >> 1) + lane;
+                float u[64];
+                tmem_ld64(tlane + TM_U + 64 * colhalf, u);
+#pragma unroll
+                for (int j = 0; j < 64; j += 8)
+                    *reinterpret_cast<uint4*>(sm + OFF_V + sw128_offset(tj, 64 * colhalf + j, 8192)) = pack8(u + j);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            named_bar_sync(kBarSerial, kSerialThreads);
+            // ---- S3: O = Qt S + P U (onto the Qt lanes of TM_C); S <- decayed S + Kb^T U
+            if (stid == 0) {
+                tc_fence_after_sync();
+                issue_mma<4, false, 0, true, 8192>(tbase + TM_C, sb + OFF_P, sb + OFF_V, ID_KxMN, true);
+                issue_mma<4, true, 8192, true, 8192>(tbase + TM_S, sb + OFF_KBAR, sb + OFF_V, ID_MNxMN, true);
+                mma_commit(&bar_os);
+            }
+            ok = mbar_wait(&bar_os, par, kTimeoutNs);
+            tc_fence_after_sync();
+            ok = named_bar_and(kBarSerial, kSerialThreads, ok);
+            if (!ok) break;
+            // ---- S4: the v tile is free: prefetch the next chunk's v; O out; S -> bf16 tile
+            if (stid == 0 && chunk + 1 < nchunks) { load_v(chunk + 1); pending = chunk + 1; }
+            if ((quarter & 1) == 0) {
+                const int r = 32 * (quarter >> 1) + lane;
+                float ov[64];
+                tmem_ld64(tlane + TM_C + 64 * colhalf, ov);   // warp-collective: every lane loads
+                if (r < nvalid) {
+                    uint4* orow = reinterpret_cast<uint4*>(p.o + (((size_t)b * T + t0 + r) * p.H + h) * kD + 64 * colhalf);
+#pragma unroll
+                    for (int j = 0; j < 64; j += 8) orow[j >> 3] = pack8(ov + j);
+                }
+            }
+            {
+                const int i = 32 * quarter + lane;
+                float sv[64];
+                tmem_ld64(tlane + TM_S + 64 * colhalf, sv);
+#pragma unroll
+                for (int j = 0; j < 64; j += 8)
+                    *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_offset(i, 64 * colhalf + j, 16384)) = pack8(sv + j);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            named_bar_sync(kBarSerial, kSerialThreads);
+        }
+        if (!ok && stid == 0) report_status(p.status, KDA_ERR_TIMEOUT);
+        if (stid == 0) {
+            mma_commit(&bar_drain_s);
+            if (!mbar_wait(&bar_drain_s, 0, kTimeoutNs)) report_status(p.status, KDA_ERR_TIMEOUT);
+            if (pending >= 0) (void)mbar_wait(&bar_v, (uint32_t)(pending & 1), kTimeoutNs);
+        }
+        named_bar_sync(kBarSerial, kSerialThreads);
+        tc_fence_after_sync();
+        if (ok && p.ST) {
+            const int i = 32 * quarter + lane;
+            float* dst = p.ST + ((size_t)bh * kD + i) * kD + 64 * colhalf;
+            float sv[64];
+            tmem_ld64(tlane + TM_S + 64 * colhalf, sv);
+#pragma unroll
+            for (int j = 0; j < 64; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
         }
     }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    if (ok && p.ST) {
-        const int i = 32 * quarter + lane;
-        float* dst = p.ST + ((size_t)bh * kD + i) * kD;
-#pragma unroll
-        for (int cb = 0; cb < 64; cb += 16) {
-            const int c0 = 64 * colhalf + cb;
-            float sv[16];
-            tmem_ld16(tlane + TM_S + c0, sv);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 16; j += 4)
-                *reinterpret_cast<float4*>(dst + c0 + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
-        }
-    }
-    tc_fence_before_sync();
-    __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, TM_COLS);
 }
 
@@ -721,6 +721,7 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 }
 
 // [B, T, H, 128] bf16 viewed as a 4-D tensor (d, H, T, B); box = 64 channels x 1 head x 64 tokens.
+// Rows past T read as zeros, which makes the tail of the last chunk an exact no-op.
 bool make_map(CUtensorMap* m, const void* ptr, int B, int T, int H) {
     auto enc = get_encode_fn();
     if (!enc) return false;
