@@ -160,6 +160,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// Same without flushing subnormal results (used for per-channel constants that multiply large factors).
+__device__ __forceinline__ float ex2_approx_sub(float x) {
+    float y;
+    asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // Load 64 TMEM columns of this warp's lanes (one wait).
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* r) {
@@ -195,7 +201,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __shared__ float s_beta[kC];
     __shared__ float s_gamma[2][kD];                   // e^{Gam_63} per channel, by chunk parity
     __shared__ __align__(16) float s_refs[4][kD];      // Gam rows 16, 31, 48, 63 (float4 access)
-    __shared__ __align__(16) float s_cst[2][4][kD];    // per block: Gam_m*log2e, e^{Gam_m}, e^{Gam_63-Gam_m}, c_off
+    __shared__ __align__(16) float s_cst[2][4][kD];    // per block: Gam_m*log2e, e^{Gam_m}, e^{Gam_63-Gam_m}, Gam_48*log2e
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3;              // TMEM lane quarter this warp may access
@@ -253,14 +259,16 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int hf = quarter & 1;                          // 32-token block of the token
         const int jr = lane;                                 // row inside the block
         const int c0 = 64 * (quarter >> 1) + 32 * colhalf;   // first of 32 channels
+        auto fetch_beta = [&](int chunk) -> float {
+            const int t = chunk * kC + ptid;
+            return (ptid < kC && t < T) ? __bfloat162float(p.beta[((size_t)b * T + t) * p.H + h]) : 0.f;
+        };
+        float beta_next = fetch_beta(0);   // beta of the next chunk, loaded a chunk ahead
         for (int chunk = 0; chunk < nchunks; ++chunk) {
             const uint32_t par = chunk & 1, ppar = par ^ 1u;
-            const int t0 = chunk * kC;
             // ---- P1: beta, L tile, Gam = L g on the tensor core
-            if (ptid < kC) {
-                const int t = t0 + ptid;
-                s_beta[ptid] = (t < T) ? __bfloat162float(p.beta[((size_t)b * T + t) * p.H + h]) : 0.f;
-            }
+            if (ptid < kC) s_beta[ptid] = beta_next;
+            if (chunk + 1 < nchunks) beta_next = fetch_beta(chunk + 1);
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int idx = ptid + kPrepThreads * e;  // 512 chunks of 8 elements
@@ -301,17 +309,17 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             ok = named_bar_and(kBarPrep, kPrepThreads, ok);
             if (!ok) break;
-            if (ptid < kD) {
-                const float g16 = s_refs[0][ptid], g48 = s_refs[2][ptid], g63 = s_refs[3][ptid];
-                s_cst[0][0][ptid] = g16 * kLog2e;
-                s_cst[0][1][ptid] = expf(g16);
-                s_cst[0][2][ptid] = expf(g63 - g16);
-                s_cst[0][3][ptid] = expf(g48 - g16);    // block-0 columns: reference 16 -> 48
-                s_cst[1][0][ptid] = g48 * kLog2e;
-                s_cst[1][1][ptid] = expf(g48);
-                s_cst[1][2][ptid] = expf(g63 - g48);
-                s_cst[1][3][ptid] = 0.f;
-                s_gamma[par][ptid] = expf(g63);
+            {
+                // per channel c and block blk: Gam_m*log2e, e^{Gam_m}, e^{Gam_63-Gam_m}, and for block 0
+                // the change of column reference 16 -> 48; e^{Gam_63} for the state decay
+                const int c = ptid & (kD - 1), blk = ptid >> 7;
+                const float g16 = s_refs[0][c], g48 = s_refs[2][c], g63 = s_refs[3][c];
+                const float gm = blk ? g48 : g16;
+                s_cst[blk][0][c] = gm * kLog2e;
+                s_cst[blk][1][c] = ex2_approx_sub(gm * kLog2e);
+                s_cst[blk][2][c] = ex2_approx_sub((g63 - gm) * kLog2e);
+                s_cst[blk][3][c] = g48 * kLog2e;      // column reference of the block-1 x block-0 rectangle
+                if (blk) s_gamma[par][c] = ex2_approx_sub(g63 * kLog2e);
             }
             // ---- P3: operand tiles (KQ may be rewritten once MMA3 of the previous chunk is done)
             if (chunk > 0) ok = mbar_wait(&bar_c, ppar, kTimeoutNs);
@@ -353,13 +361,20 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     const float qE0 = qf.x * E[0], qE1 = qf.y * E[1];
                     const float kE0 = kf.x * E[0], kE1 = kf.y * E[1];
                     const float kI0 = kf.x * Ei[0], kI1 = kf.y * Ei[1];
+                    // block-0 keys against token 48: e^{Gam_48 - Gam_j} formed directly, so it flushes
+                    // to zero only when it is itself below the fp32 range
+                    float kX0 = 0.f, kX1 = 0.f;
+                    if (hf == 0) {
+                        kX0 = kf.x * ex2_approx(co[2 * m] - G[8 * g8 + 2 * m] * kLog2e);
+                        kX1 = kf.y * ex2_approx(co[2 * m + 1] - G[8 * g8 + 2 * m + 1] * kLog2e);
+                    }
                     a1q[m] = pack_bf16x2(qE0, qE1);
                     a1k[m] = pack_bf16x2(kE0, kE1);
                     b1[m] = pack_bf16x2(kI0, kI1);
                     kqq[m] = pack_bf16x2(qE0 * cm[2 * m], qE1 * cm[2 * m + 1]);
                     kqk[m] = pack_bf16x2(kE0 * cm[2 * m], kE1 * cm[2 * m + 1]);
                     kb[4 * g8 + m] = pack_bf16x2(kI0 * ce[2 * m], kI1 * ce[2 * m + 1]);
-                    bx[m] = pack_bf16x2(kI0 * co[2 * m], kI1 * co[2 * m + 1]);
+                    bx[m] = pack_bf16x2(kX0, kX1);
                 }
                 // MMA1 operands: A rows [Qt0;Kt0;Qt1;Kt1], B rows [Kh0(16);Kh1(48);Kh0(48)]
                 *reinterpret_cast<uint4*>(sm + OFF_A1 + sw128_offset(64 * hf + jr, cc, 16384)) = make_uint4(a1q[0], a1q[1], a1q[2], a1q[3]);
@@ -382,16 +397,18 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 // raw q,k,g are consumed (Gam was read before the barrier): prefetch the next chunk
                 if (chunk + 1 < nchunks) { load_qkg(chunk + 1); pending = chunk + 1; }
             }
-            // ---- P4: P and A from TMEM, Kb tile, triangular solve, T tile
-            ok = mbar_wait(&bar_ap, par, kTimeoutNs);
-            if (ok && chunk > 0) ok = mbar_wait(&bar_os, ppar, kTimeoutNs);  // T, P, Kb released
+            // ---- P4: Kb tile, P and A from TMEM, triangular solve, T tile
+            if (chunk > 0) ok = mbar_wait(&bar_os, ppar, kTimeoutNs);  // T, P, Kb released
+            if (ok) {
+#pragma unroll
+                for (int g8 = 0; g8 < 4; ++g8)
+                    *reinterpret_cast<uint4*>(sm + OFF_KBAR + sw128_offset(tr, c0 + 8 * g8, 8192)) =
+                        make_uint4(kb[4 * g8], kb[4 * g8 + 1], kb[4 * g8 + 2], kb[4 * g8 + 3]);
+            }
+            if (ok) ok = mbar_wait(&bar_ap, par, kTimeoutNs);
             tc_fence_after_sync();
             ok = named_bar_and(kBarPrep, kPrepThreads, ok);
             if (!ok) break;
-#pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8)
-                *reinterpret_cast<uint4*>(sm + OFF_KBAR + sw128_offset(tr, c0 + 8 * g8, 8192)) =
-                    make_uint4(kb[4 * g8], kb[4 * g8 + 1], kb[4 * g8 + 2], kb[4 * g8 + 3]);
             {
                 // TMEM lane L of MMA1: quarter 0 Qt0 rows, 1 Kt0 rows, 2 Qt1 rows, 3 Kt1 rows.
                 // Columns of a row r: j < 32 from cols 0..31 (block 0) or 64..95 (block 1 rows);
@@ -571,8 +588,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const uint32_t par = chunk & 1;
             const int t0 = chunk * kC;
             const int nvalid = min(kC, T - t0);
-            // ---- S1: MMA3 = [Qt0;Kt0;Qt1;Kt1] S once the prep group has the KQ tile
-            if (stid == 0) {
+            // ---- S1: MMA3 = [Qt0;Kt0;Qt1;Kt1] S once the prep group has the KQ tile (chunk 0 here;
+            // later chunks issue it at the end of the previous chunk)
+            if (stid == 0 && chunk == 0) {
                 ok = mbar_wait(&bar_kq, par, kTimeoutNs);
                 if (ok) {
                     tc_fence_after_sync();
@@ -658,18 +676,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc_fence_after_sync();
             ok = named_bar_and(kBarSerial, kSerialThreads, ok);
             if (!ok) break;
-            // ---- S4: the v tile is free: prefetch the next chunk's v; O out; S -> bf16 tile
+            // ---- S4: the v tile is free: prefetch the next chunk's v.  S -> bf16 tile first (the next
+            // chunk's MMA3 waits on it), O read out of TMEM before MMA3 may overwrite it, stored after.
             if (stid == 0 && chunk + 1 < nchunks) { load_v(chunk + 1); pending = chunk + 1; }
-            if ((quarter & 1) == 0) {
-                const int r = 32 * (quarter >> 1) + lane;
-                float ov[64];
-                tmem_ld64(tlane + TM_C + 64 * colhalf, ov);   // warp-collective: every lane loads
-                if (r < nvalid) {
-                    uint4* orow = reinterpret_cast<uint4*>(p.o + (((size_t)b * T + t0 + r) * p.H + h) * kD + 64 * colhalf);
-#pragma unroll
-                    for (int j = 0; j < 64; j += 8) orow[j >> 3] = pack8(ov + j);
-                }
-            }
             {
                 const int i = 32 * quarter + lane;
                 float sv[64];
@@ -678,9 +687,32 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int j = 0; j < 64; j += 8)
                     *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_offset(i, 64 * colhalf + j, 16384)) = pack8(sv + j);
             }
+            uint4 opk[8];   // O row segment, already rounded to bf16
+            if ((quarter & 1) == 0) {
+                float ov[64];
+                tmem_ld64(tlane + TM_C + 64 * colhalf, ov);   // warp-collective
+#pragma unroll
+                for (int j = 0; j < 8; ++j) opk[j] = pack8(ov + 8 * j);
+            }
             fence_proxy_async_smem();
             tc_fence_before_sync();
             named_bar_sync(kBarSerial, kSerialThreads);
+            if (stid == 0 && chunk + 1 < nchunks) {
+                ok = mbar_wait(&bar_kq, par ^ 1u, kTimeoutNs);
+                if (ok) {
+                    tc_fence_after_sync();
+                    issue_mma<8, false, 16384, true, 16384>(tbase + TM_C, sb + OFF_KQ, sb + OFF_SB, ID_KxMN, false);
+                    mma_commit(&bar_c);
+                }
+            }
+            if ((quarter & 1) == 0) {
+                const int r = 32 * (quarter >> 1) + lane;
+                if (r < nvalid) {
+                    uint4* orow = reinterpret_cast<uint4*>(p.o + (((size_t)b * T + t0 + r) * p.H + h) * kD + 64 * colhalf);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) orow[j] = opk[j];
+                }
+            }
         }
         if (!ok && stid == 0) report_status(p.status, KDA_ERR_TIMEOUT);
         if (stid == 0) {

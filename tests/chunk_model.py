@@ -41,8 +41,21 @@ def _bf16(x):
     return out
 
 
-def chunk_head(q, k, v, g, beta, S0, C=64, sub=32, bf16=False):
-    """One head. q,k,g [T,dk]; v [T,dv]; beta [T]; S0 [dk,dv]. Returns (o [T,dv], S_T)."""
+def _ftz(x):
+    """Flush magnitudes below the smallest normal fp32 number to zero (as the kernel's ex2 does)."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.where(np.abs(x) < 2.0 ** -126, 0.0, x)
+
+
+def chunk_head(q, k, v, g, beta, S0, C=64, sub=32, bf16=False, offdiag_ref="block_end"):
+    """One head. q,k,g [T,dk]; v [T,dv]; beta [T]; S0 [dk,dv]. Returns (o [T,dv], S_T).
+
+    offdiag_ref: reference token of an off-diagonal block pair (R > J).  "block_end" factors at
+    the last token of block J (both factors <= 1: exact).  "row_middle" factors at the middle
+    token of block R, the same reference as the diagonal block of R, and flushes column factors
+    below the fp32 normal range to zero: this is what the tensor-core kernel does for C = 64,
+    sub = 32 (one product for the whole block row).
+    """
     T, dk = q.shape
     dv = v.shape[1]
     rnd = _bf16 if bf16 else (lambda x: x)
@@ -62,9 +75,15 @@ def chunk_head(q, k, v, g, beta, S0, C=64, sub=32, bf16=False):
             rows = slice(R * sub, (R + 1) * sub)
             for J in range(R + 1):
                 cols = slice(J * sub, (J + 1) * sub)
-                ref = Gam[R * sub + sub // 2] if J == R else Gam[J * sub + sub - 1]
-                er = np.exp(Gam[rows] - ref)
-                ej = np.exp(ref - Gam[cols])
+                if J == R or offdiag_ref == "row_middle":
+                    ref = Gam[R * sub + sub // 2]
+                else:
+                    ref = Gam[J * sub + sub - 1]
+                with np.errstate(over="ignore"):
+                    er = np.exp(Gam[rows] - ref)
+                    ej = np.exp(ref - Gam[cols])
+                if J != R and offdiag_ref == "row_middle":
+                    ej = _ftz(ej)
                 qs = rnd(qc[rows] * er)
                 ks = rnd(kc[rows] * er)
                 kh = rnd(kc[cols] * ej)
@@ -87,7 +106,7 @@ def chunk_head(q, k, v, g, beta, S0, C=64, sub=32, bf16=False):
     return o, S
 
 
-def chunk_forward(q, k, v, g, beta, S0=None, C=64, sub=32, bf16=False):
+def chunk_forward(q, k, v, g, beta, S0=None, C=64, sub=32, bf16=False, offdiag_ref="block_end"):
     """[B,T,H,*] fp64 arrays -> (o [B,T,H,dv], S_T [B,H,dk,dv])."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -97,5 +116,6 @@ def chunk_forward(q, k, v, g, beta, S0=None, C=64, sub=32, bf16=False):
         for h in range(H):
             s0 = np.zeros((dk, dv)) if S0 is None else S0[b, h]
             o[b, :, h], ST[b, h] = chunk_head(q[b, :, h], k[b, :, h], v[b, :, h], g[b, :, h],
-                                              beta[b, :, h], s0, C=C, sub=sub, bf16=bf16)
+                                              beta[b, :, h], s0, C=C, sub=sub, bf16=bf16,
+                                              offdiag_ref=offdiag_ref)
     return o, ST

@@ -46,3 +46,29 @@ def test_bf16_operands_stay_inside_tolerance(zg_mean):
     # half the 2e-2 bf16 tolerance, before the final bf16 rounding of o
     assert max_rel_err(o, o_ref) < 1e-2, max_rel_err(o, o_ref)
     assert max_rel_err(ST, ST_ref) < 1e-2, max_rel_err(ST, ST_ref)
+
+
+def adversarial_decay(T, dk, chunk=64):
+    """g = -5 on tokens 33..48 of every chunk and ~0 elsewhere: the pattern that makes the
+    block-1 x block-0 column factors e^{Gam_48 - Gam_j} underflow while nearby pair factors stay large."""
+    g = np.full((1, T, 1, dk), -1e-3)
+    for c0 in range(0, T, chunk):
+        g[:, c0 + 33:c0 + 49] = -5.0
+    return g
+
+
+@pytest.mark.parametrize("pattern", ["recipe", "adversarial", "all_minus5"])
+def test_kernel_factorisation_stays_close_to_oracle(pattern):
+    """The kernel factors the block-1 x block-0 rectangle at token 48 and flushes column factors
+    below the fp32 range.  In exact arithmetic otherwise, the dropped terms are each below
+    e^{-7.3} of a unit product; the whole effect must stay under 1e-3 of max|o| and max|S|."""
+    rng = np.random.default_rng(3)
+    q, k, v, g, beta, S0 = random_problem(rng, 1, 256, 1, 32, 32)
+    if pattern == "adversarial":
+        g = adversarial_decay(256, 32)
+    elif pattern == "all_minus5":
+        g = np.full_like(g, -5.0)
+    o_ref, ST_ref = oracle.forward(q, k, v, g, beta, S0, nthreads=2)
+    o, ST = chunk_forward(q, k, v, g, beta, S0, C=64, sub=32, offdiag_ref="row_middle")
+    assert max_rel_err(o, o_ref) < 1e-3, max_rel_err(o, o_ref)
+    assert max_rel_err(ST, ST_ref) < 1e-3, max_rel_err(ST, ST_ref)

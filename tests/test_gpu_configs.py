@@ -38,13 +38,19 @@ def oracle_heads(inputs, heads):
 
 
 @pytest.mark.parametrize("T", [64, 128, 191, 320, 1000])
-@pytest.mark.parametrize("regime", ["recipe", "worst_decay", "no_decay"])
+@pytest.mark.parametrize("regime", ["recipe", "worst_decay", "no_decay", "adversarial"])
 def test_tc_matches_oracle(T, regime):
     q, k, v, g, beta, S0 = make_prefill_inputs(2, T, 3, 128, 128, "bf16", seed=T, s0_std=0.1, device=DEV)
     if regime == "worst_decay":
         g = torch.full_like(g, -5.0)
     elif regime == "no_decay":
         g = (g * 0.01).contiguous()      # long memory: the state carries across many chunks
+    elif regime == "adversarial":
+        # g = -5 on tokens 33..48 of every chunk, ~0 elsewhere: column factors of the block-1 x
+        # block-0 rectangle underflow while nearby pair factors stay of order one
+        g = torch.full_like(g, -1e-3)
+        for c0 in range(0, T, 64):
+            g[:, c0 + 33:c0 + 49] = -5.0
     o, ST = kda.kda_forward_chunked(q, k, v, g, beta, S0, impl="tcgen05")
     torch.cuda.synchronize()
     assert kda.kda_get_device_status() == 0
