@@ -134,6 +134,24 @@ KDA_API const char* kda_status_string(int status);
 /* kda_version -- library version as major*10000 + minor*100 + patch. */
 KDA_API int kda_version(void);
 
+/*
+ * kda_debug_set_wait_fault -- TEST HOOK for the device-side timeout path (not for production).
+ *
+ * The tensor-core prefill coordinates its two warp groups with mbarrier waits, each bounded
+ * in wall time (2 s by default); a wait that runs out sets the status word to
+ * KDA_ERR_TIMEOUT, lets every warp of the CTA leave its loop, drains the outstanding
+ * tensor-core and TMA work, frees the tensor memory and returns.  Nothing traps, faults or
+ * hangs, and the CUDA context stays usable.
+ *
+ *   mode 1: subsequent tcgen05 prefill launches skip the first hand-off from the operand
+ *           warps to the recurrence warps, so a wait is guaranteed to run out; every wait
+ *           is limited to timeout_ns (1 ms .. 10 s).  Outputs of such launches are undefined.
+ *   mode 0: normal operation (the timeout_ns argument is ignored; 2 s limit).
+ *
+ * Process-wide setting, read at launch.  Returns KDA_OK or KDA_ERR_INVALID_ARG.
+ */
+KDA_API int kda_debug_set_wait_fault(int mode, unsigned long long timeout_ns);
+
 #ifdef __cplusplus
 }
 #endif

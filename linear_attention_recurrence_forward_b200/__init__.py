@@ -25,6 +25,7 @@ __all__ = [
     "kda_decode_step",
     "kda_get_device_status",
     "kda_status_string",
+    "kda_debug_set_wait_fault",
     "KdaError",
     "lib",
     "LIB_PATH",
@@ -77,6 +78,8 @@ def lib() -> ctypes.CDLL:
         L.kda_status_string.restype = ctypes.c_char_p
         L.kda_version.argtypes = []
         L.kda_version.restype = I
+        L.kda_debug_set_wait_fault.argtypes = [I, ctypes.c_ulonglong]
+        L.kda_debug_set_wait_fault.restype = I
         _lib = L
     return _lib
 
@@ -168,3 +171,10 @@ def kda_get_device_status(stream=None, device=None) -> int:
     """Synchronise the stream, then return and clear the device status word (0 = OK)."""
     with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
         return int(lib().kda_get_device_status(_stream_handle(stream)))
+
+
+def kda_debug_set_wait_fault(mode: int, timeout_ns: int = 0) -> None:
+    """Test hook: mode 1 makes tensor-core prefill launches time out a bounded device wait."""
+    rc = lib().kda_debug_set_wait_fault(int(mode), int(timeout_ns))
+    if rc != 0:
+        raise KdaError("kda_debug_set_wait_fault", rc)

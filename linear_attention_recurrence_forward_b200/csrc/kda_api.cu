@@ -3,6 +3,7 @@
 // Everything here runs on the host before a launch; nothing is enqueued unless every
 // check passes.  The kernels themselves live in kda_decode.cu, kda_prefill_simt.cu and
 // kda_prefill_tc.cu.
+#include <atomic>
 #include <mutex>
 #include <stdint.h>
 
@@ -15,7 +16,11 @@ __device__ int g_kda_status_word = 0;
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per device-side wait
 std::mutex g_mutex;
+// Wait-timeout test hook (kda_debug_set_wait_fault); read at every tensor-core prefill launch.
+std::atomic<int> g_skip_handoff{0};
+std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
 int* g_status_addr[kMaxDevices] = {nullptr};
 
 int* status_word_for_current_device() {
@@ -90,7 +95,8 @@ int forward_impl(const void* q, const void* k, const void* v, const void* g, con
         return KDA_ERR_INVALID_ARG;
     int rc = validate_prefill(q, k, v, g, beta, S0, o, ST, B, T, H, dk, dv, dtype);
     if (rc != KDA_OK) return rc;
-    kda::PrefillArgs a{q, k, v, g, beta, S0, o, ST, B, T, H, dk, dv, dtype, nullptr};
+    kda::PrefillArgs a{q, k, v, g, beta, S0, o, ST, B, T, H, dk, dv, dtype, nullptr,
+                       g_timeout_ns.load(), g_skip_handoff.load()};
     const bool tc_ok = kda::prefill_tc_supports(a);
     if (impl == KDA_IMPL_TCGEN05 && !tc_ok) return KDA_ERR_UNSUPPORTED;
     if (T == 0) {
@@ -175,5 +181,13 @@ const char* kda_status_string(int status) {
 }
 
 int kda_version(void) { return 100; }
+
+int kda_debug_set_wait_fault(int mode, unsigned long long timeout_ns) {
+    if (mode != 0 && mode != 1) return KDA_ERR_INVALID_ARG;
+    if (mode == 1 && (timeout_ns < 1000000ull || timeout_ns > 10000000000ull)) return KDA_ERR_INVALID_ARG;
+    g_skip_handoff.store(mode);
+    g_timeout_ns.store(mode ? timeout_ns : kDefaultTimeoutNs);
+    return KDA_OK;
+}
 
 }  // extern "C"

@@ -22,6 +22,8 @@ struct PrefillArgs {
     int B, T, H, dk, dv;
     int dtype;        // kda_dtype
     int* status;      // device status word
+    unsigned long long timeout_ns;  // limit of every device-side wait
+    int skip_handoff;               // test hook: 1 = the prep group never signals its first hand-off
 };
 
 struct DecodeArgs {

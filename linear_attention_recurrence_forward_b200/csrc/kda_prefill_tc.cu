@@ -53,7 +53,6 @@ constexpr int kThreads = 512;   // 16 warps
 constexpr int kPrepThreads = 256;
 constexpr int kSerialThreads = 256;
 constexpr uint32_t kBarPrep = 1, kBarSerial = 2;   // named hardware barriers
-constexpr uint64_t kTimeoutNs = 2000000000ull;      // bounded waits: 2 s
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
 constexpr uint32_t OFF_RAW_Q = 0;           // TMA destination, bf16 [64 tok][128], 2 boxes of 8 KB
@@ -100,6 +99,8 @@ struct TcParams {
     __nv_bfloat16* o;
     float* ST;
     int* status;
+    unsigned long long timeout_ns;  // limit of every mbarrier wait
+    int skip_handoff;               // test hook: never signal the first KQ hand-off
     int B, T, H;
 };
 
@@ -281,7 +282,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             fence_proxy_async_smem();
             if (ptid == 0) {
-                ok = mbar_wait(&bar_qkg, par, kTimeoutNs);
+                ok = mbar_wait(&bar_qkg, par, p.timeout_ns);
                 if (ok) pending = -1;
             }
             ok = named_bar_and(kBarPrep, kPrepThreads, ok);
@@ -296,7 +297,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 mma_commit(&bar_g);
             }
             // ---- P2: Gam rows and per-channel constants
-            ok = mbar_wait(&bar_g, par, kTimeoutNs);
+            ok = mbar_wait(&bar_g, par, p.timeout_ns);
             tc_fence_after_sync();
             float G[32];
             tmem_ld16(tlane + TM_P + c0, G);
@@ -322,7 +323,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 if (blk) s_gamma[par][c] = ex2_approx_sub(g63 * kLog2e);
             }
             // ---- P3: operand tiles (KQ may be rewritten once MMA3 of the previous chunk is done)
-            if (chunk > 0) ok = mbar_wait(&bar_c, ppar, kTimeoutNs);
+            if (chunk > 0) ok = mbar_wait(&bar_c, ppar, p.timeout_ns);
             ok = named_bar_and(kBarPrep, kPrepThreads, ok);
             if (!ok) break;
             uint32_t kb[16];  // Kb of this token row, written once the previous chunk released the tile
@@ -391,21 +392,21 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             named_bar_sync(kBarPrep, kPrepThreads);
             if (ptid == 0) {
                 tc_fence_after_sync();
-                mbar_arrive(&bar_kq);  // KQ of this chunk is ready for MMA3
+                if (!(p.skip_handoff && chunk == 0)) mbar_arrive(&bar_kq);  // KQ of this chunk is ready for MMA3
                 issue_mma<8, false, 16384, false, 12288>(tbase + TM_P, sb + OFF_A1, sb + OFF_BB, ID_MMA1, false);
                 mma_commit(&bar_ap);
                 // raw q,k,g are consumed (Gam was read before the barrier): prefetch the next chunk
                 if (chunk + 1 < nchunks) { load_qkg(chunk + 1); pending = chunk + 1; }
             }
             // ---- P4: Kb tile, P and A from TMEM, triangular solve, T tile
-            if (chunk > 0) ok = mbar_wait(&bar_os, ppar, kTimeoutNs);  // T, P, Kb released
+            if (chunk > 0) ok = mbar_wait(&bar_os, ppar, p.timeout_ns);  // T, P, Kb released
             if (ok) {
 #pragma unroll
                 for (int g8 = 0; g8 < 4; ++g8)
                     *reinterpret_cast<uint4*>(sm + OFF_KBAR + sw128_offset(tr, c0 + 8 * g8, 8192)) =
                         make_uint4(kb[4 * g8], kb[4 * g8 + 1], kb[4 * g8 + 2], kb[4 * g8 + 3]);
             }
-            if (ok) ok = mbar_wait(&bar_ap, par, kTimeoutNs);
+            if (ok) ok = mbar_wait(&bar_ap, par, p.timeout_ns);
             tc_fence_after_sync();
             ok = named_bar_and(kBarPrep, kPrepThreads, ok);
             if (!ok) break;
@@ -550,8 +551,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // drain: no MMA or TMA issued by this group may still be in flight
         if (ptid == 0) {
             mma_commit(&bar_drain_p);
-            if (!mbar_wait(&bar_drain_p, 0, kTimeoutNs)) report_status(p.status, KDA_ERR_TIMEOUT);
-            if (pending >= 0) (void)mbar_wait(&bar_qkg, (uint32_t)(pending & 1), kTimeoutNs);
+            if (!mbar_wait(&bar_drain_p, 0, p.timeout_ns)) report_status(p.status, KDA_ERR_TIMEOUT);
+            if (pending >= 0) (void)mbar_wait(&bar_qkg, (uint32_t)(pending & 1), p.timeout_ns);
         }
     } else {
         // ====================================================================== serial group
@@ -591,7 +592,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // ---- S1: MMA3 = [Qt0;Kt0;Qt1;Kt1] S once the prep group has the KQ tile (chunk 0 here;
             // later chunks issue it at the end of the previous chunk)
             if (stid == 0 && chunk == 0) {
-                ok = mbar_wait(&bar_kq, par, kTimeoutNs);
+                ok = mbar_wait(&bar_kq, par, p.timeout_ns);
                 if (ok) {
                     tc_fence_after_sync();
                     issue_mma<8, false, 16384, true, 16384>(tbase + TM_C, sb + OFF_KQ, sb + OFF_SB, ID_KxMN, false);
@@ -599,8 +600,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
             }
             // Y = V - Kt S (Kt rows sit in lanes 32-63 and 96-127), in place over v
-            if (ok) ok = mbar_wait(&bar_c, par, kTimeoutNs);
-            if (ok) ok = mbar_wait(&bar_v, par, kTimeoutNs);
+            if (ok) ok = mbar_wait(&bar_c, par, p.timeout_ns);
+            if (ok) ok = mbar_wait(&bar_v, par, p.timeout_ns);
             tc_fence_after_sync();
             ok = named_bar_and(kBarSerial, kSerialThreads, ok);
             if (!ok) break;
@@ -629,7 +630,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             named_bar_sync(kBarSerial, kSerialThreads);
             // ---- S2: MMA4 U = T Y once the prep group has T, P, Kb; decay the state meanwhile
             if (stid == 0) {
-                ok = mbar_wait(&bar_tpk, par, kTimeoutNs);
+                ok = mbar_wait(&bar_tpk, par, p.timeout_ns);
                 if (ok) {
                     tc_fence_after_sync();
                     issue_mma<4, false, 0, true, 8192>(tbase + TM_U, sb + OFF_T, sb + OFF_V, ID_KxMN, false);
@@ -649,7 +650,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int cb = 0; cb < 64; cb += 16) tmem_st16(tlane + TM_S + 64 * colhalf + cb, sv + cb);
                 tmem_wait_st();
             }
-            ok = mbar_wait(&bar_u, par, kTimeoutNs);
+            ok = mbar_wait(&bar_u, par, p.timeout_ns);
             tc_fence_after_sync();
             ok = named_bar_and(kBarSerial, kSerialThreads, ok);
             if (!ok) break;
@@ -672,7 +673,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 issue_mma<4, true, 8192, true, 8192>(tbase + TM_S, sb + OFF_KBAR, sb + OFF_V, ID_MNxMN, true);
                 mma_commit(&bar_os);
             }
-            ok = mbar_wait(&bar_os, par, kTimeoutNs);
+            ok = mbar_wait(&bar_os, par, p.timeout_ns);
             tc_fence_after_sync();
             ok = named_bar_and(kBarSerial, kSerialThreads, ok);
             if (!ok) break;
@@ -698,7 +699,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc_fence_before_sync();
             named_bar_sync(kBarSerial, kSerialThreads);
             if (stid == 0 && chunk + 1 < nchunks) {
-                ok = mbar_wait(&bar_kq, par ^ 1u, kTimeoutNs);
+                ok = mbar_wait(&bar_kq, par ^ 1u, p.timeout_ns);
                 if (ok) {
                     tc_fence_after_sync();
                     issue_mma<8, false, 16384, true, 16384>(tbase + TM_C, sb + OFF_KQ, sb + OFF_SB, ID_KxMN, false);
@@ -717,8 +718,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (!ok && stid == 0) report_status(p.status, KDA_ERR_TIMEOUT);
         if (stid == 0) {
             mma_commit(&bar_drain_s);
-            if (!mbar_wait(&bar_drain_s, 0, kTimeoutNs)) report_status(p.status, KDA_ERR_TIMEOUT);
-            if (pending >= 0) (void)mbar_wait(&bar_v, (uint32_t)(pending & 1), kTimeoutNs);
+            if (!mbar_wait(&bar_drain_s, 0, p.timeout_ns)) report_status(p.status, KDA_ERR_TIMEOUT);
+            if (pending >= 0) (void)mbar_wait(&bar_v, (uint32_t)(pending & 1), p.timeout_ns);
         }
         named_bar_sync(kBarSerial, kSerialThreads);
         tc_fence_after_sync();
@@ -792,7 +793,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
         !make_map(&mg, a.g, a.B, a.T, a.H) || !make_map(&mv, a.v, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
     TcParams prm{static_cast<const __nv_bfloat16*>(a.beta), a.S0, static_cast<__nv_bfloat16*>(a.o), a.ST,
-                 a.status, a.B, a.T, a.H};
+                 a.status, a.timeout_ns, a.skip_handoff, a.B, a.T, a.H};
     kda_prefill_tc_kernel<<<(unsigned)((size_t)a.B * a.H), kThreads, SMEM_DYN, s>>>(mq, mk, mg, mv, prm);
     return cudaGetLastError();
 }

@@ -137,3 +137,11 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     with pytest.raises(ImportError):
         mod.lib()
     importlib.reload(kda)
+
+
+def test_wait_fault_hook_validates_arguments(L):
+    assert L.kda_debug_set_wait_fault(2, 10_000_000) == INVALID
+    assert L.kda_debug_set_wait_fault(1, 10) == INVALID            # below 1 ms
+    assert L.kda_debug_set_wait_fault(1, 20_000_000_000) == INVALID  # above 10 s
+    assert L.kda_debug_set_wait_fault(1, 20_000_000) == OK
+    assert L.kda_debug_set_wait_fault(0, 0) == OK
