@@ -56,13 +56,21 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def kernel_source_sha():
+KERNEL_SOURCES = {
+    "prefill_tc": ("kda_prefill_tc.cu", "sm100_ptx.cuh", "kda_internal.cuh"),
+    "prefill_simt": ("kda_prefill_simt.cu", "kda_internal.cuh"),
+    "decode": ("kda_decode.cu", "kda_internal.cuh"),
+}
+
+
+def kernel_source_sha(kernel_tag):
+    """Short hash of the source files a kernel is built from (a recorded ncu figure is valid only
+    while they are unchanged)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_attention_recurrence_forward_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in KERNEL_SOURCES[kernel_tag]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -71,7 +79,7 @@ def recorded_traffic(kernel_tag):
     prof = os.path.join(ROOT, "profiles")
     if not os.path.isdir(prof):
         return None
-    sha = kernel_source_sha()
+    sha = kernel_source_sha(kernel_tag)
     for name in sorted(os.listdir(prof)):
         if not name.endswith(".md"):
             continue
@@ -186,6 +194,36 @@ def run_reference(args):
     return 0
 
 
+def measure_e2e(kda, dist, world, dev, stream, args, q, k, v, g, beta, S0, o):
+    """Prefill through the public API with pinned host inputs copied in and o copied out, per step."""
+    import torch
+    P = PREFILL
+    host_in = [t.to("cpu").pin_memory() for t in (q, k, v, g, beta)]
+    host_s0 = S0.to("cpu").pin_memory()
+    host_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    e2e_steps = max(1, min(args.steps, 3))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        dq, dk_, dv_, dg, db = (t.to(dev, non_blocking=True) for t in host_in)
+        ds0 = host_s0.to(dev, non_blocking=True)
+        oo, _ = kda.kda_forward_chunked(dq, dk_, dv_, dg, db, ds0, stream=stream)
+        host_o.copy_(oo, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    h2d = sum(t.numel() * t.element_size() for t in host_in) + host_s0.numel() * 4
+    d2h = host_o.numel() * host_o.element_size()
+    return {"value": world * P["B"] * P["T"] / (e2e_ms.item() / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "note": "prefill through kda_forward_chunked with pinned host inputs copied in and o copied out"}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -264,28 +302,10 @@ def run_ours(args):
     total_ms, prefill_sum, decode_sum = tm.tolist()
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
-    host_in = [t.to("cpu").pin_memory() for t in (q, k, v, g, beta)]
-    host_s0 = S0.to("cpu").pin_memory()
-    host_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    e2e_steps = max(1, min(args.steps, 3))
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        dq, dk_, dv_, dg, db = (t.to(dev, non_blocking=True) for t in host_in)
-        ds0 = host_s0.to(dev, non_blocking=True)
-        oo, _ = kda.kda_forward_chunked(dq, dk_, dv_, dg, db, ds0, stream=stream)
-        host_o.copy_(oo, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    h2d = sum(t.numel() * t.element_size() for t in host_in) + host_s0.numel() * 4
-    d2h = host_o.numel() * host_o.element_size()
-
+    if args.no_e2e:
+        e2e = None
+    else:
+        e2e = measure_e2e(kda, dist, world, dev, stream, args, q, k, v, g, beta, S0, o)
     tokens_per_prefill = P["B"] * P["T"]
     value = world * tokens_per_prefill * args.steps / (prefill_sum / 1e3)
     states = D["batch"] * D["H"]
@@ -327,9 +347,7 @@ def run_ours(args):
                                 "frac": dec_achieved / peak, "alg_bytes_per_launch": db_,
                                 "traffic": recorded_traffic("decode")}},
         "cpu_baseline": cpu,
-        "e2e": {"value": world * tokens_per_prefill / (e2e_ms.item() / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "note": "prefill through kda_forward_chunked with pinned host inputs copied in and o copied out"},
+        "e2e": e2e,
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
     }
@@ -347,9 +365,18 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-shape", default=None, metavar="B,T,H",
+                    help="override the prefill workload (profiling small cases); the line is then not the headline")
+    ap.add_argument("--decode-batch", type=int, default=None, help="override the decode batch (profiling)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.prefill_shape:
+        B, T, H = (int(x) for x in args.prefill_shape.split(","))
+        PREFILL.update(B=B, T=T, H=H, name=f"prefill_b{B}_t{T}_h{H}")
+    if args.decode_batch:
+        DECODE.update(batch=args.decode_batch, name=f"decode_b{args.decode_batch}_h{DECODE['H']}")
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
