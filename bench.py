@@ -194,6 +194,21 @@ def run_reference(args):
     return 0
 
 
+def max_over_ranks(values, device, world):
+    """Element-wise max of per-rank timings (every rank gets the result); identity for one rank."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def weak_scaling_throughput(units_per_rank, world, steps, seconds):
+    """Whole-job throughput: every rank processed units_per_rank per step; time is the max over ranks."""
+    return world * units_per_rank * steps / seconds
+
+
 def measure_e2e(kda, dist, world, dev, stream, args, q, k, v, g, beta, S0, o):
     """Prefill through the public API with pinned host inputs copied in and o copied out, per step."""
     import torch
@@ -214,12 +229,10 @@ def measure_e2e(kda, dist, world, dev, stream, args, q, k, v, g, beta, S0, o):
         host_o.copy_(oo, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], dev, world)
     h2d = sum(t.numel() * t.element_size() for t in host_in) + host_s0.numel() * 4
     d2h = host_o.numel() * host_o.element_size()
-    return {"value": world * P["B"] * P["T"] / (e2e_ms.item() / 1e3), "unit": "tokens/s",
+    return {"value": weak_scaling_throughput(P["B"] * P["T"], world, 1, e2e_ms / 1e3), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "note": "prefill through kda_forward_chunked with pinned host inputs copied in and o copied out"}
 
@@ -296,10 +309,7 @@ def run_ours(args):
     total_ms = t_start.elapsed_time(t_end)
     prefill_ms = [e[0].elapsed_time(e[1]) for e in evs]
     decode_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    tm = torch.tensor([total_ms, sum(prefill_ms), sum(decode_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-    total_ms, prefill_sum, decode_sum = tm.tolist()
+    total_ms, prefill_sum, decode_sum = max_over_ranks([total_ms, sum(prefill_ms), sum(decode_ms)], dev, world)
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
     if args.no_e2e:
@@ -307,9 +317,9 @@ def run_ours(args):
     else:
         e2e = measure_e2e(kda, dist, world, dev, stream, args, q, k, v, g, beta, S0, o)
     tokens_per_prefill = P["B"] * P["T"]
-    value = world * tokens_per_prefill * args.steps / (prefill_sum / 1e3)
+    value = weak_scaling_throughput(tokens_per_prefill, world, args.steps, prefill_sum / 1e3)
     states = D["batch"] * D["H"]
-    decode_states_per_s = world * states * args.steps / (decode_sum / 1e3)
+    decode_states_per_s = weak_scaling_throughput(states, world, args.steps, decode_sum / 1e3)
     peak, peak_kind = measured_peaks()
     pb = prefill_alg_bytes(P["B"], P["T"], P["H"], P["dk"], P["dv"])
     prefill_launch_ms = prefill_sum / args.steps
