@@ -252,6 +252,10 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int ptid = tid;                               // 0..255
         int pending = -1;                                   // chunk whose q,k,g loads are in flight
         if (ptid == 0) { load_qkg(0); pending = 0; }
+        // T's strictly upper 16x16 blocks stay zero for the whole sequence: clear the tile once
+        for (int idx = ptid; idx < 512; idx += kPrepThreads)
+            *reinterpret_cast<uint4*>(sm + OFF_T + sw128_offset(tp_row(idx >> 3), (idx & 7) * 8, 8192)) =
+                make_uint4(0u, 0u, 0u, 0u);
         float* AF = reinterpret_cast<float*>(sm + OFF_AF);
         float* XF = reinterpret_cast<float*>(sm + OFF_X);
         float* XT = reinterpret_cast<float*>(sm + OFF_XT);
@@ -260,15 +264,18 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int hf = quarter & 1;                          // 32-token block of the token
         const int jr = lane;                                 // row inside the block
         const int c0 = 64 * (quarter >> 1) + 32 * colhalf;   // first of 32 channels
-        auto fetch_beta = [&](int chunk) -> float {
+        // beta of the next chunk, loaded a chunk ahead as raw bf16 bits (converted only when it is
+        // stored, so the load's latency is never waited for)
+        const unsigned short* beta_bits = reinterpret_cast<const unsigned short*>(p.beta);
+        auto fetch_beta = [&](int chunk) -> unsigned short {
             const int t = chunk * kC + ptid;
-            return (ptid < kC && t < T) ? __bfloat162float(p.beta[((size_t)b * T + t) * p.H + h]) : 0.f;
+            return (ptid < kC && t < T) ? beta_bits[((size_t)b * T + t) * p.H + h] : (unsigned short)0;
         };
-        float beta_next = fetch_beta(0);   // beta of the next chunk, loaded a chunk ahead
+        unsigned short beta_next = fetch_beta(0);
         for (int chunk = 0; chunk < nchunks; ++chunk) {
             const uint32_t par = chunk & 1, ppar = par ^ 1u;
             // ---- P1: beta, L tile, Gam = L g on the tensor core
-            if (ptid < kC) s_beta[ptid] = beta_next;
+            if (ptid < kC) s_beta[ptid] = __uint_as_float((uint32_t)beta_next << 16);
             if (chunk + 1 < nchunks) beta_next = fetch_beta(chunk + 1);
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -482,6 +489,12 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
                 for (int r = 0; r < 16; r += 4)
                     *reinterpret_cast<float4*>(XT + (o0 + c) * kLd + o0 + r) = make_float4(x[r], x[r + 1], x[r + 2], x[r + 3]);
+                // T = X Diag(beta): this diagonal block's column c
+                const float bc = s_beta[o0 + c];
+#pragma unroll
+                for (int r = 0; r < 16; ++r)
+                    *reinterpret_cast<__nv_bfloat16*>(sm + OFF_T + sw128_offset(tp_row(o0 + r), o0 + c, 8192)) =
+                        __float2bfloat16_rn(x[r] * bc);
             }
             named_bar_sync(kBarPrep, kPrepThreads);
             // X_RJ = -X_RR sum_{L=J}^{R-1} A_RL X_LJ by block distance d = R - J on warp-level bf16
@@ -523,25 +536,15 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         XT[(col + 1) * kLd + 16 * R + g4] = -x[1];
                         XT[col * kLd + 16 * R + g4 + 8] = -x[2];
                         XT[(col + 1) * kLd + 16 * R + g4 + 8] = -x[3];
+                        // T = X Diag(beta) for these entries
+                        const float b0 = s_beta[col], b1 = s_beta[col + 1];
+                        *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(16 * R + g4), col, 8192)) =
+                            pack_bf16x2(-x[0] * b0, -x[1] * b1);
+                        *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(16 * R + g4 + 8), col, 8192)) =
+                            pack_bf16x2(-x[2] * b0, -x[3] * b1);
                     }
                     named_bar_sync(kBarPrep, kPrepThreads);
                 }
-            }
-            // T = X Diag(beta), bf16, K-major (K = 64 tokens); strictly upper blocks are 0
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int idx = ptid + kPrepThreads * e;  // 512 chunks of 8
-                const int r = idx >> 3, j = (idx & 7) * 8;
-                uint4 pk = make_uint4(0u, 0u, 0u, 0u);
-                if ((j >> 4) <= (r >> 4)) {
-                    const float4 xa = *reinterpret_cast<const float4*>(XF + r * kLd + j);
-                    const float4 xb = *reinterpret_cast<const float4*>(XF + r * kLd + j + 4);
-                    pk.x = pack_bf16x2(xa.x * s_beta[j + 0], xa.y * s_beta[j + 1]);
-                    pk.y = pack_bf16x2(xa.z * s_beta[j + 2], xa.w * s_beta[j + 3]);
-                    pk.z = pack_bf16x2(xb.x * s_beta[j + 4], xb.y * s_beta[j + 5]);
-                    pk.w = pack_bf16x2(xb.z * s_beta[j + 6], xb.w * s_beta[j + 7]);
-                }
-                *reinterpret_cast<uint4*>(sm + OFF_T + sw128_offset(tp_row(r), j, 8192)) = pk;
             }
             fence_proxy_async_smem();
             named_bar_sync(kBarPrep, kPrepThreads);
