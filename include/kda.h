@@ -104,6 +104,29 @@ KDA_API int kda_forward_chunked_impl(const void* q, const void* k, const void* v
                              struct CUstream_st* stream);
 
 /*
+ * kda_forward_chunked_states -- kda_forward_chunked that also writes the state after every
+ * `interval` tokens: the boundaries from which a prefix cache resumes the recurrence
+ * (podcast show-notes (scripod.com), outline item 5.3.1 "KDA-Aware Prefix Cache Management";
+ * the channel post on the K3 report (t.iss.one), online-inference paragraph: prefixes are
+ * reused at 512-token boundaries).
+ *
+ *   S_mid    : [B, H, n_mid, dk, dv] fp32 output, n_mid = T / interval (integer division):
+ *              S_mid[b][h][n] is the state after the first (n+1)*interval tokens of (b, h),
+ *              the same values a kda_forward_chunked over those tokens returns as S_T.
+ *              Must not overlap any other argument.  May be NULL only when n_mid == 0.
+ *   interval : a positive multiple of 64 (the prefill's chunk length).
+ *   impl     : kda_impl, as for kda_forward_chunked_impl.
+ *
+ * Every other argument, layout and rule as kda_forward_chunked; o and S_T are the values it
+ * would produce.  Returns KDA_ERR_INVALID_ARG for interval <= 0, KDA_ERR_UNSUPPORTED for an
+ * interval that is not a multiple of 64.
+ */
+KDA_API int kda_forward_chunked_states(const void* q, const void* k, const void* v, const void* g,
+                               const void* beta, const float* S0, void* o, float* S_T,
+                               float* S_mid, int interval, int B, int T, int H, int dk, int dv,
+                               int dtype, int impl, struct CUstream_st* stream);
+
+/*
  * kda_decode_step -- one token for every (b, h), state updated in place.
  *
  * Same recurrence with T = 1 (the memory-bound state read-modify-write of decoding):

@@ -6,6 +6,7 @@ these functions raise.
 
     from linear_attention_recurrence_forward_b200 import kda_forward_chunked, kda_decode_step
     o, S_T = kda_forward_chunked(q, k, v, g, beta, S0)        # prefill, torch CUDA tensors
+    o, S_T, S_mid = kda_forward_chunked_states(q, k, v, g, beta, S0, interval=512)
     o = kda_decode_step(q, k, v, g, beta, S)                   # one token, S updated in place
 
 Layouts (contiguous): q, k, g [B, T, H, dk]; v, o [B, T, H, dv]; beta [B, T, H];
@@ -22,6 +23,7 @@ import torch
 
 __all__ = [
     "kda_forward_chunked",
+    "kda_forward_chunked_states",
     "kda_decode_step",
     "kda_get_device_status",
     "kda_status_string",
@@ -70,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.kda_forward_chunked.restype = I
         L.kda_forward_chunked_impl.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P]
         L.kda_forward_chunked_impl.restype = I
+        L.kda_forward_chunked_states.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]
+        L.kda_forward_chunked_states.restype = I
         L.kda_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P]
         L.kda_decode_step.restype = I
         L.kda_get_device_status.argtypes = [P]
@@ -142,6 +146,46 @@ def kda_forward_chunked(q, k, v, g, beta, S0=None, *, o=None, S_T=None, return_s
     if rc != 0:
         raise KdaError("kda_forward_chunked", rc)
     return o, S_T
+
+
+def kda_forward_chunked_states(q, k, v, g, beta, S0=None, *, interval: int = 512, o=None, S_T=None,
+                               S_mid=None, impl: str = "auto", stream=None):
+    """Prefill that also returns the state after every `interval` tokens (a multiple of 64).
+
+    Returns (o, S_T, S_mid) with S_mid [B, H, T // interval, dk, dv] fp32: S_mid[:, :, n] is the
+    state after the first (n + 1) * interval tokens.
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    if dt not in DTYPE:
+        raise ValueError(f"unsupported dtype {dt}")
+    for name, t, shape in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("v", v, (B, T, H, dv)),
+                           ("g", g, (B, T, H, dk)), ("beta", beta, (B, T, H))):
+        _check(t, name, shape, dt, dev)
+    if S0 is not None:
+        _check(S0, "S0", (B, H, dk, dv), torch.float32, dev)
+    n_mid = T // interval if interval > 0 else 0
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    else:
+        _check(o, "o", (B, T, H, dv), dt, dev)
+    if S_T is None:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    else:
+        _check(S_T, "S_T", (B, H, dk, dv), torch.float32, dev)
+    if S_mid is None:
+        S_mid = torch.empty((B, H, n_mid, dk, dv), dtype=torch.float32, device=dev)
+    else:
+        _check(S_mid, "S_mid", (B, H, n_mid, dk, dv), torch.float32, dev)
+    with torch.cuda.device(dev):
+        rc = lib().kda_forward_chunked_states(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                                              _ptr(o), _ptr(S_T), _ptr(S_mid) if n_mid > 0 else None,
+                                              int(interval), B, T, H, dk, dv, DTYPE[dt], IMPL[impl],
+                                              _stream_handle(stream))
+    if rc != 0:
+        raise KdaError("kda_forward_chunked_states", rc)
+    return o, S_T, S_mid
 
 
 def kda_decode_step(q, k, v, g, beta, S, *, o=None, stream=None):

@@ -88,15 +88,45 @@ int validate_prefill(const void* q, const void* k, const void* v, const void* g,
     return KDA_OK;
 }
 
+// The intermediate-state output: interval, size, alignment, and no overlap with anything else.
+int validate_states(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                    const float* S0, const void* o, const float* ST, const float* S_mid, int interval,
+                    int B, int T, int H, int dk, int dv, int dtype, int* n_mid_out) {
+    if (interval <= 0) return KDA_ERR_INVALID_ARG;
+    if (interval % 64 != 0) return KDA_ERR_UNSUPPORTED;
+    const int n_mid = T / interval;
+    *n_mid_out = n_mid;
+    if (n_mid == 0) return KDA_OK;
+    if (!S_mid) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(S_mid)) return KDA_ERR_MISALIGNED;
+    const size_t es = elem_size(dtype);
+    const size_t n_tok = (size_t)B * T * H;
+    const size_t sbytes = (size_t)B * H * dk * dv * sizeof(float);
+    const Range rm = range_of(S_mid, sbytes * (size_t)n_mid);
+    const Range others[] = {range_of(q, n_tok * dk * es), range_of(k, n_tok * dk * es),
+                            range_of(v, n_tok * dv * es), range_of(g, n_tok * dk * es),
+                            range_of(beta, n_tok * es), range_of(o, n_tok * dv * es),
+                            range_of(S0, S0 ? sbytes : 0), range_of(ST, ST ? sbytes : 0)};
+    for (const Range& r : others)
+        if (overlaps(rm, r)) return KDA_ERR_INVALID_ARG;
+    return KDA_OK;
+}
+
 int forward_impl(const void* q, const void* k, const void* v, const void* g, const void* beta,
                  const float* S0, void* o, float* ST, int B, int T, int H, int dk, int dv, int dtype,
-                 int impl, cudaStream_t stream) {
+                 int impl, cudaStream_t stream, float* S_mid = nullptr, int interval = 0) {
     if (impl != KDA_IMPL_AUTO && impl != KDA_IMPL_TCGEN05 && impl != KDA_IMPL_SIMT)
         return KDA_ERR_INVALID_ARG;
     int rc = validate_prefill(q, k, v, g, beta, S0, o, ST, B, T, H, dk, dv, dtype);
     if (rc != KDA_OK) return rc;
+    int n_mid = 0;
+    if (interval != 0 || S_mid) {
+        rc = validate_states(q, k, v, g, beta, S0, o, ST, S_mid, interval, B, T, H, dk, dv, dtype, &n_mid);
+        if (rc != KDA_OK) return rc;
+    }
     kda::PrefillArgs a{q, k, v, g, beta, S0, o, ST, B, T, H, dk, dv, dtype, nullptr,
-                       g_timeout_ns.load(), g_skip_handoff.load()};
+                       g_timeout_ns.load(), g_skip_handoff.load(), n_mid > 0 ? S_mid : nullptr,
+                       interval, n_mid};
     const bool tc_ok = kda::prefill_tc_supports(a);
     if (impl == KDA_IMPL_TCGEN05 && !tc_ok) return KDA_ERR_UNSUPPORTED;
     if (T == 0) {
@@ -130,6 +160,15 @@ int kda_forward_chunked_impl(const void* q, const void* k, const void* v, const 
                              const void* beta, const float* S0, void* o, float* S_T, int B, int T,
                              int H, int dk, int dv, int dtype, int impl, struct CUstream_st* stream) {
     return forward_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, dtype, impl, stream);
+}
+
+int kda_forward_chunked_states(const void* q, const void* k, const void* v, const void* g,
+                               const void* beta, const float* S0, void* o, float* S_T,
+                               float* S_mid, int interval, int B, int T, int H, int dk, int dv,
+                               int dtype, int impl, struct CUstream_st* stream) {
+    if (interval <= 0) return KDA_ERR_INVALID_ARG;
+    return forward_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, dtype, impl, stream, S_mid,
+                        interval);
 }
 
 int kda_decode_step(const void* q, const void* k, const void* v, const void* g, const void* beta,

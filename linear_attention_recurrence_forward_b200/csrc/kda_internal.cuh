@@ -24,6 +24,9 @@ struct PrefillArgs {
     int* status;      // device status word
     unsigned long long timeout_ns;  // limit of every device-side wait
     int skip_handoff;               // test hook: 1 = the prep group never signals its first hand-off
+    float* S_mid;                   // states every `interval` tokens [B, H, n_mid, dk, dv], or null
+    int interval;                   // multiple of 64 when S_mid is set
+    int n_mid;                      // T / interval when S_mid is set, else 0
 };
 
 struct DecodeArgs {

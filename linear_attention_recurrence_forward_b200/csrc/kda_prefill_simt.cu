@@ -24,7 +24,8 @@ template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kSimtThreads)
 kda_prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                         const Tin* __restrict__ g, const Tin* __restrict__ beta,
-                        const float* S0, Tin* __restrict__ o, float* ST, int T, int H) {
+                        const float* S0, Tin* __restrict__ o, float* ST, int T, int H,
+                        float* S_mid, int interval, int n_mid) {
     constexpr int RPT = DK / kRpp;  // rows per thread (4 or 2)
     constexpr int NW = kSimtThreads / 32;
     constexpr int NSLICE = DV / kSlice;
@@ -122,6 +123,15 @@ kda_prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, co
             const float kr = ks[buf][rg + j * kRpp];
             s[j].x += kr * u.x; s[j].y += kr * u.y; s[j].z += kr * u.z; s[j].w += kr * u.w;
         }
+        // the state after a multiple of the interval
+        if (n_mid > 0 && (t + 1) % interval == 0) {
+            const size_t base = bh * (size_t)n_mid + (size_t)((t + 1) / interval - 1);
+#pragma unroll
+            for (int j = 0; j < RPT; ++j) {
+                const int r = rg + j * kRpp;
+                __stcs(reinterpret_cast<float4*>(S_mid + (base * DK + r) * DV + col0 + 4 * c4), s[j]);
+            }
+        }
     }
     if (ST) {
 #pragma unroll
@@ -138,7 +148,7 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s) {
     kda_prefill_simt_kernel<Tin, DK, DV><<<grid, kSimtThreads, 0, s>>>(
         static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
         static_cast<const Tin*>(a.g), static_cast<const Tin*>(a.beta), a.S0, static_cast<Tin*>(a.o),
-        a.ST, a.T, a.H);
+        a.ST, a.T, a.H, a.S_mid, a.interval, a.n_mid);
     return cudaGetLastError();
 }
 

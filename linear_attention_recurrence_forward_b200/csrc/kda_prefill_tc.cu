@@ -53,6 +53,7 @@ constexpr int kThreads = 512;   // 16 warps
 constexpr int kPrepThreads = 256;
 constexpr int kSerialThreads = 256;
 constexpr uint32_t kBarPrep = 1, kBarSerial = 2;   // named hardware barriers
+constexpr int kIssuer = 0;                         // prep thread that issues its TMA loads and MMAs
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
 constexpr uint32_t OFF_RAW_Q = 0;           // TMA destination, bf16 [64 tok][128], 2 boxes of 8 KB
@@ -62,7 +63,6 @@ constexpr uint32_t OFF_V = 49152;           // v, then Y = V - Kt S, then U (MN-
 constexpr uint32_t OFF_AP = 65536;          // prep operand region (56 KB)
 constexpr uint32_t OFF_A1 = OFF_AP;                 // [Qt0;Kt0;Qt1;Kt1] block-middle refs, K-major, 2 x 16 KB
 constexpr uint32_t OFF_BB = OFF_AP + 32768;         // [Kh0(16);Kh1(48);Kh0(48)], K-major, 96 rows, 2 x 12 KB
-constexpr uint32_t OFF_L = OFF_AP + 8192;           // chunk start: lower-triangular ones (8 KB)
 constexpr int kLd = 68;                              // padded row stride (floats) of the solve matrices
 constexpr int kLdS = 20;
 constexpr uint32_t OFF_AF = OFF_AP;                  // after MMA1: A (fp32 64 x kLd)
@@ -84,10 +84,9 @@ static_assert(OFF_BB + 2 * 12288 <= OFF_KQ, "BB overlaps KQ");
 constexpr uint32_t TM_S = 0;     // S (dk lanes x dv columns), fp32 master state
 constexpr uint32_t TM_C = 128;   // MMA3: lanes 0-31 Qt0 S, 32-63 Kt0 S, 64-95 Qt1 S, 96-127 Kt1 S; + P U
 constexpr uint32_t TM_U = 256;   // MMA4: U at lanes 0-31 (tokens 0-31) and 64-95 (tokens 32-63)
-constexpr uint32_t TM_P = 384;   // prep: Gam (128 columns), then MMA1 (96 columns)
+constexpr uint32_t TM_P = 384;   // prep: MMA1 (96 columns)
 constexpr uint32_t TM_COLS = 512;
 
-constexpr uint32_t ID_G = idesc_bf16_f32(128, 64, false, true);
 constexpr uint32_t ID_MMA1 = idesc_bf16_f32(128, 96, false, false);
 constexpr uint32_t ID_KxMN = idesc_bf16_f32(128, 128, false, true);
 constexpr uint32_t ID_MNxMN = idesc_bf16_f32(128, 128, true, true);
@@ -101,9 +100,17 @@ struct TcParams {
     int* status;
     unsigned long long timeout_ns;  // limit of every mbarrier wait
     int skip_handoff;               // test hook: never signal the first KQ hand-off
+    float* S_mid;                   // state after every `interval` tokens, or null
+    int interval, n_mid;
     int B, T, H;
 };
 
+// Element-wise bf16x2 product, rounded to nearest even.
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&p);
@@ -196,13 +203,13 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t sb = smem_u32(sm);
 
     // TMA / MMA completion barriers (one phase per chunk) and prep -> serial hand-offs.
-    __shared__ uint64_t bar_qkg, bar_v, bar_g, bar_ap, bar_c, bar_u, bar_os, bar_kq, bar_tpk;
+    __shared__ uint64_t bar_qkg, bar_v, bar_ap, bar_c, bar_u, bar_os, bar_kq, bar_tpk;
     __shared__ uint64_t bar_drain_p, bar_drain_s;
     __shared__ uint32_t tmem_base_s;
-    __shared__ float s_beta[kC];
-    __shared__ float s_gamma[2][kD];                   // e^{Gam_63} per channel, by chunk parity
-    __shared__ __align__(16) float s_refs[4][kD];      // Gam rows 16, 31, 48, 63 (float4 access)
-    __shared__ __align__(16) float s_cst[2][4][kD];    // per block: Gam_m*log2e, e^{Gam_m}, e^{Gam_63-Gam_m}, Gam_48*log2e
+    __shared__ __align__(16) float s_beta[kC];
+    __shared__ __align__(16) float s_gamma[2][kD];     // e^{Gam_63} per channel, by chunk parity (float2 stores)
+    __shared__ __align__(16) float s_refs[4][kD];      // Gam rows 16, 31, 48, 63
+    __shared__ __align__(16) float s_qsum[4][kD];      // g summed over each 16-token quarter
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3;              // TMEM lane quarter this warp may access
@@ -214,7 +221,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const int nchunks = (T + kC - 1) / kC;
 
     if (tid == 0) {
-        mbar_init(&bar_qkg, 1); mbar_init(&bar_v, 1); mbar_init(&bar_g, 1); mbar_init(&bar_ap, 1);
+        mbar_init(&bar_qkg, 1); mbar_init(&bar_v, 1); mbar_init(&bar_ap, 1);
         mbar_init(&bar_c, 1); mbar_init(&bar_u, 1); mbar_init(&bar_os, 1); mbar_init(&bar_kq, 1);
         mbar_init(&bar_tpk, 1); mbar_init(&bar_drain_p, 1); mbar_init(&bar_drain_s, 1);
         fence_mbar_init();
@@ -250,8 +257,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (is_prep) {
         // ====================================================================== prep group
         const int ptid = tid;                               // 0..255
-        int pending = -1;                                   // chunk whose q,k,g loads are in flight
-        if (ptid == 0) { load_qkg(0); pending = 0; }
+        int pending = -1;                                   // chunk whose q,k,g loads are in flight (issuer)
+        if (ptid == kIssuer) { load_qkg(0); pending = 0; }
         // T's strictly upper 16x16 blocks stay zero for the whole sequence: clear the tile once
         for (int idx = ptid; idx < 512; idx += kPrepThreads)
             *reinterpret_cast<uint4*>(sm + OFF_T + sw128_offset(tp_row(idx >> 3), (idx & 7) * 8, 8192)) =
@@ -259,11 +266,11 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         float* AF = reinterpret_cast<float*>(sm + OFF_AF);
         float* XF = reinterpret_cast<float*>(sm + OFF_X);
         float* XT = reinterpret_cast<float*>(sm + OFF_XT);
-        // token row / channel range of this thread in the element-wise step
-        const int tr = 32 * (quarter & 1) + lane;            // token
-        const int hf = quarter & 1;                          // 32-token block of the token
-        const int jr = lane;                                 // row inside the block
-        const int c0 = 64 * (quarter >> 1) + 32 * colhalf;   // first of 32 channels
+        // this thread's part of the Gam scan and of the element-wise step: channels ch0, ch0 + 1 of the
+        // 16 tokens of quarter tq (a warp covers 64 channels of one quarter)
+        const int tq = warp >> 1;
+        const int hq = tq >> 1;                              // 32-token block (reference token 16 or 48)
+        const int ch0 = 64 * (warp & 1) + 2 * lane;
         // beta of the next chunk, loaded a chunk ahead as raw bf16 bits (converted only when it is
         // stored, so the load's latency is never waited for)
         const unsigned short* beta_bits = reinterpret_cast<const unsigned short*>(p.beta);
@@ -274,130 +281,116 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         unsigned short beta_next = fetch_beta(0);
         for (int chunk = 0; chunk < nchunks; ++chunk) {
             const uint32_t par = chunk & 1, ppar = par ^ 1u;
-            // ---- P1: beta, L tile, Gam = L g on the tensor core
+            // ---- P1: beta; this chunk's q, k, g
             if (ptid < kC) s_beta[ptid] = __uint_as_float((uint32_t)beta_next << 16);
             if (chunk + 1 < nchunks) beta_next = fetch_beta(chunk + 1);
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int idx = ptid + kPrepThreads * e;  // 512 chunks of 8 elements
-                const int r = idx >> 3, j0 = (idx & 7) * 8;
-                uint32_t w[4];
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    w[m] = ((j0 + 2 * m <= r) ? 0x3F80u : 0u) | ((j0 + 2 * m + 1 <= r) ? 0x3F800000u : 0u);
-                *reinterpret_cast<uint4*>(sm + OFF_L + sw128_offset(r, j0, 8192)) = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            fence_proxy_async_smem();
-            if (ptid == 0) {
+            if (ptid == kIssuer) {
                 ok = mbar_wait(&bar_qkg, par, p.timeout_ns);
                 if (ok) pending = -1;
             }
             ok = named_bar_and(kBarPrep, kPrepThreads, ok);
             if (!ok) break;
-            if (ptid == 0) {
-                tc_fence_after_sync();
-                // channels 0..63 into lanes 0..63 (A rows 64..127 read other smem),
-                // channels 64..127 into lanes 64..127 (A rows 0..63 read other smem)
-                issue_mma<4, false, 0, true, 8192>(tbase + TM_P, sb + OFF_L, sb + OFF_RAW_G, ID_G, false);
-                issue_mma<4, false, 0, true, 8192>(tbase + TM_P + 64, sb + OFF_L - 8192, sb + OFF_RAW_G + 8192,
-                                                   ID_G, false);
-                mma_commit(&bar_g);
-            }
-            // ---- P2: Gam rows and per-channel constants
-            ok = mbar_wait(&bar_g, par, p.timeout_ns);
-            tc_fence_after_sync();
-            float G[32];
-            tmem_ld16(tlane + TM_P + c0, G);
-            tmem_ld16(tlane + TM_P + c0 + 16, G + 16);
-            tmem_wait_ld();
-            if (lane == 16 || lane == 31) {
-                float* dst = &s_refs[2 * hf + (lane == 31)][c0];
-#pragma unroll
-                for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(G[e], G[e + 1], G[e + 2], G[e + 3]);
-            }
-            ok = named_bar_and(kBarPrep, kPrepThreads, ok);
-            if (!ok) break;
+            // ---- P2: Gam = in-chunk prefix sum of g in fp32: the running sum over this quarter,
+            // then the totals of the quarters before it
+            float gam[16][2];
             {
-                // per channel c and block blk: Gam_m*log2e, e^{Gam_m}, e^{Gam_63-Gam_m}, and for block 0
-                // the change of column reference 16 -> 48; e^{Gam_63} for the state decay
-                const int c = ptid & (kD - 1), blk = ptid >> 7;
-                const float g16 = s_refs[0][c], g48 = s_refs[2][c], g63 = s_refs[3][c];
-                const float gm = blk ? g48 : g16;
-                s_cst[blk][0][c] = gm * kLog2e;
-                s_cst[blk][1][c] = ex2_approx_sub(gm * kLog2e);
-                s_cst[blk][2][c] = ex2_approx_sub((g63 - gm) * kLog2e);
-                s_cst[blk][3][c] = g48 * kLog2e;      // column reference of the block-1 x block-0 rectangle
-                if (blk) s_gamma[par][c] = ex2_approx_sub(g63 * kLog2e);
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_G + sw128_offset(16 * tq + i, ch0, 8192));
+                    a0 += __uint_as_float(w << 16);
+                    a1 += __uint_as_float(w & 0xFFFF0000u);
+                    gam[i][0] = a0;
+                    gam[i][1] = a1;
+                }
+                *reinterpret_cast<float2*>(&s_qsum[tq][ch0]) = make_float2(a0, a1);
+            }
+            named_bar_sync(kBarPrep, kPrepThreads);
+            {
+                float c0s = 0.f, c1s = 0.f;
+#pragma unroll 1
+                for (int qq = 0; qq < tq; ++qq) {
+                    const float2 s2 = *reinterpret_cast<const float2*>(&s_qsum[qq][ch0]);
+                    c0s += s2.x;
+                    c1s += s2.y;
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) { gam[i][0] += c0s; gam[i][1] += c1s; }
+            }
+            if (tq & 1) {
+                // tokens 16 and 31 (quarter 1), 48 and 63 (quarter 3); e^{Gam_63} for the state decay
+                *reinterpret_cast<float2*>(&s_refs[2 * hq][ch0]) = make_float2(gam[0][0], gam[0][1]);
+                *reinterpret_cast<float2*>(&s_refs[2 * hq + 1][ch0]) = make_float2(gam[15][0], gam[15][1]);
+                if (hq)
+                    *reinterpret_cast<float2*>(&s_gamma[par][ch0]) =
+                        make_float2(ex2_approx_sub(gam[15][0] * kLog2e), ex2_approx_sub(gam[15][1] * kLog2e));
             }
             // ---- P3: operand tiles (KQ may be rewritten once MMA3 of the previous chunk is done)
             if (chunk > 0) ok = mbar_wait(&bar_c, ppar, p.timeout_ns);
             ok = named_bar_and(kBarPrep, kPrepThreads, ok);
             if (!ok) break;
-            uint32_t kb[16];  // Kb of this token row, written once the previous chunk released the tile
-#pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
-                const int cc = c0 + 8 * g8;
-                const uint32_t roff = sw128_offset(tr, cc, 8192);
-                const uint4 qraw = *reinterpret_cast<const uint4*>(sm + OFF_RAW_Q + roff);
-                const uint4 kraw = *reinterpret_cast<const uint4*>(sm + OFF_RAW_K + roff);
-                float gmL[8], cm[8], ce[8], co[8];
-#pragma unroll
-                for (int u = 0; u < 8; u += 4) {
-                    const float4 x0 = *reinterpret_cast<const float4*>(&s_cst[hf][0][cc + u]);
-                    const float4 x1 = *reinterpret_cast<const float4*>(&s_cst[hf][1][cc + u]);
-                    const float4 x2 = *reinterpret_cast<const float4*>(&s_cst[hf][2][cc + u]);
-                    const float4 x3 = *reinterpret_cast<const float4*>(&s_cst[hf][3][cc + u]);
-                    gmL[u] = x0.x; gmL[u + 1] = x0.y; gmL[u + 2] = x0.z; gmL[u + 3] = x0.w;
-                    cm[u] = x1.x; cm[u + 1] = x1.y; cm[u + 2] = x1.z; cm[u + 3] = x1.w;
-                    ce[u] = x2.x; ce[u + 1] = x2.y; ce[u + 2] = x2.z; ce[u + 3] = x2.w;
-                    co[u] = x3.x; co[u + 1] = x3.y; co[u + 2] = x3.z; co[u + 3] = x3.w;
-                }
-                const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qraw);
-                const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kraw);
-                uint32_t a1q[4], a1k[4], b1[4], kqk[4], kqq[4], bx[4];
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const float2 qf = __bfloat1622float2(q2[m]);
-                    const float2 kf = __bfloat1622float2(k2[m]);
-                    float E[2], Ei[2];
+            uint32_t kb[16];  // Kb of these tokens, written once the previous chunk released the tile
+            {
+                // per channel, against the block's reference token m: Gam_m*log2e, e^{Gam_63-Gam_m},
+                // e^{Gam_m} (bf16 pair), and for block 0 the two factors of the column change to
+                // token 48, e^{Gam_31-Gam_16} and e^{Gam_48-Gam_31}.  Each factor spans at most 17
+                // tokens, so at g >= -5 it stays a normal float.
+                float gmL[2], ce[2], em[2], f1[2] = {0.f, 0.f}, f2[2] = {0.f, 0.f};
+                {
+                    const float2 r16 = *reinterpret_cast<const float2*>(&s_refs[0][ch0]);
+                    const float2 r31 = *reinterpret_cast<const float2*>(&s_refs[1][ch0]);
+                    const float2 r48 = *reinterpret_cast<const float2*>(&s_refs[2][ch0]);
+                    const float2 r63 = *reinterpret_cast<const float2*>(&s_refs[3][ch0]);
+                    const float g16[2] = {r16.x, r16.y}, g31[2] = {r31.x, r31.y};
+                    const float g48[2] = {r48.x, r48.y}, g63[2] = {r63.x, r63.y};
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const float xl = fmaf(G[8 * g8 + 2 * m + u], kLog2e, -gmL[2 * m + u]);
-                        E[u] = ex2_approx(xl);
-                        Ei[u] = ex2_approx(-xl);
+                        const float gm = hq ? g48[u] : g16[u];
+                        gmL[u] = gm * kLog2e;
+                        ce[u] = ex2_approx_sub((g63[u] - gm) * kLog2e);
+                        em[u] = ex2_approx_sub(gm * kLog2e);
+                        if (hq == 0) {
+                            f1[u] = ex2_approx_sub((g31[u] - g16[u]) * kLog2e);
+                            f2[u] = ex2_approx_sub((g48[u] - g31[u]) * kLog2e);
+                        }
                     }
-                    const float qE0 = qf.x * E[0], qE1 = qf.y * E[1];
-                    const float kE0 = kf.x * E[0], kE1 = kf.y * E[1];
-                    const float kI0 = kf.x * Ei[0], kI1 = kf.y * Ei[1];
-                    // block-0 keys against token 48: e^{Gam_48 - Gam_j} formed directly, so it flushes
-                    // to zero only when it is itself below the fp32 range
-                    float kX0 = 0.f, kX1 = 0.f;
-                    if (hf == 0) {
-                        kX0 = kf.x * ex2_approx(co[2 * m] - G[8 * g8 + 2 * m] * kLog2e);
-                        kX1 = kf.y * ex2_approx(co[2 * m + 1] - G[8 * g8 + 2 * m + 1] * kLog2e);
-                    }
-                    a1q[m] = pack_bf16x2(qE0, qE1);
-                    a1k[m] = pack_bf16x2(kE0, kE1);
-                    b1[m] = pack_bf16x2(kI0, kI1);
-                    kqq[m] = pack_bf16x2(qE0 * cm[2 * m], qE1 * cm[2 * m + 1]);
-                    kqk[m] = pack_bf16x2(kE0 * cm[2 * m], kE1 * cm[2 * m + 1]);
-                    kb[4 * g8 + m] = pack_bf16x2(kI0 * ce[2 * m], kI1 * ce[2 * m + 1]);
-                    bx[m] = pack_bf16x2(kX0, kX1);
                 }
-                // MMA1 operands: A rows [Qt0;Kt0;Qt1;Kt1], B rows [Kh0(16);Kh1(48);Kh0(48)]
-                *reinterpret_cast<uint4*>(sm + OFF_A1 + sw128_offset(64 * hf + jr, cc, 16384)) = make_uint4(a1q[0], a1q[1], a1q[2], a1q[3]);
-                *reinterpret_cast<uint4*>(sm + OFF_A1 + sw128_offset(64 * hf + 32 + jr, cc, 16384)) = make_uint4(a1k[0], a1k[1], a1k[2], a1k[3]);
-                *reinterpret_cast<uint4*>(sm + OFF_BB + sw128_offset(tr, cc, 12288)) = make_uint4(b1[0], b1[1], b1[2], b1[3]);
-                if (hf == 0)
-                    *reinterpret_cast<uint4*>(sm + OFF_BB + sw128_offset(64 + jr, cc, 12288)) = make_uint4(bx[0], bx[1], bx[2], bx[3]);
-                // MMA3 operand: the same row order against the chunk start
-                *reinterpret_cast<uint4*>(sm + OFF_KQ + sw128_offset(64 * hf + jr, cc, 16384)) = make_uint4(kqq[0], kqq[1], kqq[2], kqq[3]);
-                *reinterpret_cast<uint4*>(sm + OFF_KQ + sw128_offset(64 * hf + 32 + jr, cc, 16384)) = make_uint4(kqk[0], kqk[1], kqk[2], kqk[3]);
+                const uint32_t cmb = pack_bf16x2(em[0], em[1]);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int t = 16 * tq + i;
+                    const int rq = 64 * hq + (t & 31), rk = rq + 32;   // MMA1 rows [Qt0;Kt0;Qt1;Kt1]
+                    const uint32_t qw = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_Q + sw128_offset(t, ch0, 8192));
+                    const uint32_t kw = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_K + sw128_offset(t, ch0, 8192));
+                    const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xFFFF0000u);
+                    const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
+                    const float x0 = fmaf(gam[i][0], kLog2e, -gmL[0]);
+                    const float x1 = fmaf(gam[i][1], kLog2e, -gmL[1]);
+                    const float E0 = ex2_approx(x0), E1 = ex2_approx(x1);
+                    const float I0 = ex2_approx(-x0), I1 = ex2_approx(-x1);
+                    const float kI0 = k0 * I0, kI1 = k1 * I1;
+                    const uint32_t a1q = pack_bf16x2(q0 * E0, q1 * E1);
+                    const uint32_t a1k = pack_bf16x2(k0 * E0, k1 * E1);
+                    // MMA1 operands: A rows [Qt0;Kt0;Qt1;Kt1], B rows [Kh0(16);Kh1(48);Kh0(48)]
+                    *reinterpret_cast<uint32_t*>(sm + OFF_A1 + sw128_offset(rq, ch0, 16384)) = a1q;
+                    *reinterpret_cast<uint32_t*>(sm + OFF_A1 + sw128_offset(rk, ch0, 16384)) = a1k;
+                    *reinterpret_cast<uint32_t*>(sm + OFF_BB + sw128_offset(t, ch0, 12288)) = pack_bf16x2(kI0, kI1);
+                    // block-0 keys against token 48: k e^{Gam_16-Gam_j} e^{Gam_31-Gam_16} e^{Gam_48-Gam_31},
+                    // multiplied left to right; the middle product k e^{Gam_31-Gam_j} never exceeds |k|,
+                    // so a factor flushes to zero only when the exact product is below the fp32 range
+                    if (hq == 0)
+                        *reinterpret_cast<uint32_t*>(sm + OFF_BB + sw128_offset(64 + t, ch0, 12288)) =
+                            pack_bf16x2((kI0 * f1[0]) * f2[0], (kI1 * f1[1]) * f2[1]);
+                    // MMA3 operand, the same rows against the chunk start: the bf16 tile times bf16 e^{Gam_m}
+                    *reinterpret_cast<uint32_t*>(sm + OFF_KQ + sw128_offset(rq, ch0, 16384)) = mul_bf16x2(a1q, cmb);
+                    *reinterpret_cast<uint32_t*>(sm + OFF_KQ + sw128_offset(rk, ch0, 16384)) = mul_bf16x2(a1k, cmb);
+                    kb[i] = pack_bf16x2(kI0 * ce[0], kI1 * ce[1]);
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
             named_bar_sync(kBarPrep, kPrepThreads);
-            if (ptid == 0) {
+            if (ptid == kIssuer) {
                 tc_fence_after_sync();
                 if (!(p.skip_handoff && chunk == 0)) mbar_arrive(&bar_kq);  // KQ of this chunk is ready for MMA3
                 issue_mma<8, false, 16384, false, 12288>(tbase + TM_P, sb + OFF_A1, sb + OFF_BB, ID_MMA1, false);
@@ -409,9 +402,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (chunk > 0) ok = mbar_wait(&bar_os, ppar, p.timeout_ns);  // T, P, Kb released
             if (ok) {
 #pragma unroll
-                for (int g8 = 0; g8 < 4; ++g8)
-                    *reinterpret_cast<uint4*>(sm + OFF_KBAR + sw128_offset(tr, c0 + 8 * g8, 8192)) =
-                        make_uint4(kb[4 * g8], kb[4 * g8 + 1], kb[4 * g8 + 2], kb[4 * g8 + 3]);
+                for (int i = 0; i < 16; ++i)
+                    *reinterpret_cast<uint32_t*>(sm + OFF_KBAR + sw128_offset(16 * tq + i, ch0, 8192)) = kb[i];
             }
             if (ok) ok = mbar_wait(&bar_ap, par, p.timeout_ns);
             tc_fence_after_sync();
@@ -463,7 +455,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     }
                 }
             }
-            tc_fence_before_sync();  // the next chunk's Gam product reuses these TMEM columns
+            tc_fence_before_sync();  // the next chunk's MMA1 reuses these TMEM columns
             named_bar_sync(kBarPrep, kPrepThreads);
             // diagonal 16x16 blocks of X = (I + A)^-1 by forward substitution, one lane per column:
             // x_r = e_c[r] - sum_{l<r} A[r][l] x_l (the strictly upper entries of A are stored as 0)
@@ -552,7 +544,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         if (!ok && ptid == 0) report_status(p.status, KDA_ERR_TIMEOUT);
         // drain: no MMA or TMA issued by this group may still be in flight
-        if (ptid == 0) {
+        if (ptid == kIssuer) {
             mma_commit(&bar_drain_p);
             if (!mbar_wait(&bar_drain_p, 0, p.timeout_ns)) report_status(p.status, KDA_ERR_TIMEOUT);
             if (pending >= 0) (void)mbar_wait(&bar_qkg, (uint32_t)(pending & 1), p.timeout_ns);
@@ -690,6 +682,13 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
                 for (int j = 0; j < 64; j += 8)
                     *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_offset(i, 64 * colhalf + j, 16384)) = pack8(sv + j);
+                // the state after a multiple of the interval (only a full chunk can end on one)
+                if (p.n_mid > 0 && t0 + kC <= T && (t0 + kC) % p.interval == 0) {
+                    float* dst = p.S_mid + (((size_t)bh * p.n_mid + (t0 + kC) / p.interval - 1) * kD + i) * kD + 64 * colhalf;
+#pragma unroll
+                    for (int j = 0; j < 64; j += 4)
+                        __stcs(reinterpret_cast<float4*>(dst + j), make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]));
+                }
             }
             uint4 opk[8];   // O row segment, already rounded to bf16
             if ((quarter & 1) == 0) {
@@ -796,7 +795,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
         !make_map(&mg, a.g, a.B, a.T, a.H) || !make_map(&mv, a.v, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
     TcParams prm{static_cast<const __nv_bfloat16*>(a.beta), a.S0, static_cast<__nv_bfloat16*>(a.o), a.ST,
-                 a.status, a.timeout_ns, a.skip_handoff, a.B, a.T, a.H};
+                 a.status, a.timeout_ns, a.skip_handoff, a.S_mid, a.interval, a.n_mid, a.B, a.T, a.H};
     kda_prefill_tc_kernel<<<(unsigned)((size_t)a.B * a.H), kThreads, SMEM_DYN, s>>>(mq, mk, mg, mv, prm);
     return cudaGetLastError();
 }

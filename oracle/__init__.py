@@ -58,6 +58,9 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     L = ctypes.c_long
     lib.kda_oracle_forward.argtypes = [P, P, P, P, P, P, P, P, L, L, L, L, L, ctypes.c_int]
     lib.kda_oracle_forward.restype = ctypes.c_int
+    if hasattr(lib, "kda_oracle_forward_states"):
+        lib.kda_oracle_forward_states.argtypes = [P, P, P, P, P, P, P, P, P, L, L, L, L, L, L, ctypes.c_int]
+        lib.kda_oracle_forward_states.restype = ctypes.c_int
     lib.kda_oracle_decode_step.argtypes = [P, P, P, P, P, P, P, L, L, L, L, ctypes.c_int]
     lib.kda_oracle_decode_step.restype = ctypes.c_int
     lib.kda_oracle_max_threads.argtypes = []
@@ -110,6 +113,29 @@ def forward(q, k, v, g, beta, S0=None, nthreads: int = 0, lib: ctypes.CDLL = Non
     if rc != 0:
         raise ValueError(f"oracle rejected the shapes (rc={rc})")
     return o, ST
+
+
+def forward_states(q, k, v, g, beta, S0=None, interval: int = 512, nthreads: int = 0,
+                   lib: ctypes.CDLL = None):
+    """forward() that also returns the state after every `interval` tokens.
+
+    Returns (o [B,T,H,dv], S_T [B,H,dk,dv], S_mid [B,H,T//interval,dk,dv]) in fp64; S_mid[:, :, n]
+    is the state after the first (n+1)*interval tokens.
+    """
+    lib = lib or _get_lib()
+    q, k, v, g, beta, S0 = (to_f64(x) for x in (q, k, v, g, beta, S0))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert interval > 0
+    o = np.zeros((B, T, H, dv), np.float64)
+    ST = np.zeros((B, H, dk, dv), np.float64)
+    S_mid = np.zeros((B, H, T // interval, dk, dv), np.float64)
+    rc = lib.kda_oracle_forward_states(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                                       _ptr(o), _ptr(ST), _ptr(S_mid), int(interval), B, T, H, dk, dv,
+                                       int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the shapes (rc={rc})")
+    return o, ST, S_mid
 
 
 def decode_step(q, k, v, g, beta, S: np.ndarray, nthreads: int = 0, lib: ctypes.CDLL = None):

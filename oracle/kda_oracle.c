@@ -34,6 +34,7 @@
  *
  * Layouts (row-major, contiguous): q,k,g [B,T,H,dk]; v,o [B,T,H,dv]; beta [B,T,H];
  * S0, ST [B,H,dk,dv].  S0 may be NULL (zero state), ST may be NULL (not returned).
+ * Intermediate states (kda_oracle_forward_states): S_mid [B,H,T/interval,dk,dv].
  * Decode: q,k,g [B,H,dk]; v,o [B,H,dv]; beta [B,H]; S [B,H,dk,dv] updated in place.
  */
 #include <math.h>
@@ -68,12 +69,23 @@ static void oracle_token(double* S, const double* q, const double* k, const doub
         for (c = 0; c < dv; ++c) o[c] += S[i * dv + c] * q[i];
 }
 
-int kda_oracle_forward(const double* q, const double* k, const double* v, const double* g,
-                       const double* beta, const double* S0, double* o, double* ST,
-                       long B, long T, long H, long dk, long dv, int nthreads)
+/*
+ * The whole sequence for every (b, h).  When S_mid is not NULL it also records the state
+ * after every `interval` tokens: the boundaries at which a prefix cache can resume the
+ * recurrence (podcast show-notes (scripod.com), outline item 5.3.1 "KDA-Aware Prefix Cache
+ * Management"; the channel post on the K3 report (t.iss.one), online-inference paragraph:
+ * prefixes are reused at 512-token boundaries).  S_mid is [B, H, T / interval, dk, dv] and
+ * entry n holds the state after tokens 1 .. (n+1)*interval.
+ */
+static int oracle_forward_impl(const double* q, const double* k, const double* v, const double* g,
+                               const double* beta, const double* S0, double* o, double* ST,
+                               double* S_mid, long interval, long B, long T, long H, long dk,
+                               long dv, int nthreads)
 {
     long bh;
+    const long n_mid = (S_mid && interval > 0) ? T / interval : 0;
     if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+    if (S_mid && interval <= 0) return -1;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
 #pragma omp parallel for schedule(dynamic, 1)
@@ -88,11 +100,31 @@ int kda_oracle_forward(const double* q, const double* k, const double* v, const 
             long row = (b * T + t) * H + h;
             oracle_token(S, q + row * dk, k + row * dk, v + row * dv, g + row * dk, beta[row],
                          o + row * dv, p, dk, dv);
+            if (n_mid > 0 && (t + 1) % interval == 0)
+                memcpy(S_mid + (bh * n_mid + (t + 1) / interval - 1) * dk * dv, S,
+                       sizeof(double) * (size_t)(dk * dv));
         }
         if (ST) memcpy(ST + bh * dk * dv, S, sizeof(double) * (size_t)(dk * dv));
         free(S);
     }
     return 0;
+}
+
+int kda_oracle_forward(const double* q, const double* k, const double* v, const double* g,
+                       const double* beta, const double* S0, double* o, double* ST,
+                       long B, long T, long H, long dk, long dv, int nthreads)
+{
+    return oracle_forward_impl(q, k, v, g, beta, S0, o, ST, NULL, 0, B, T, H, dk, dv, nthreads);
+}
+
+int kda_oracle_forward_states(const double* q, const double* k, const double* v, const double* g,
+                              const double* beta, const double* S0, double* o, double* ST,
+                              double* S_mid, long interval, long B, long T, long H, long dk,
+                              long dv, int nthreads)
+{
+    if (!S_mid) return -1;
+    return oracle_forward_impl(q, k, v, g, beta, S0, o, ST, S_mid, interval, B, T, H, dk, dv,
+                               nthreads);
 }
 
 int kda_oracle_decode_step(const double* q, const double* k, const double* v, const double* g,

@@ -54,7 +54,8 @@ def chunk_head(q, k, v, g, beta, S0, C=64, sub=32, bf16=False, offdiag_ref="bloc
     the last token of block J (both factors <= 1: exact).  "row_middle" factors at the middle
     token of block R, the same reference as the diagonal block of R, and flushes column factors
     below the fp32 normal range to zero: this is what the tensor-core kernel does for C = 64,
-    sub = 32 (one product for the whole block row).
+    sub = 32 (one product for the whole block row).  The kernel builds those column factors from
+    in-range pieces, so it flushes no more than this model does.
     """
     T, dk = q.shape
     dv = v.shape[1]
@@ -93,8 +94,16 @@ def chunk_head(q, k, v, g, beta, S0, C=64, sub=32, bf16=False, offdiag_ref="bloc
             P = np.where(np.tril(np.ones((C, C), bool)), P, 0.0)
             A = np.where(np.tril(np.ones((C, C), bool), -1), A, 0.0) * bc[:, None]
         Tm = np.linalg.solve(np.eye(C) + A, np.diag(bc))
-        Kt = rnd(kc * np.exp(Gam))
-        Qt = rnd(qc * np.exp(Gam))
+        if bf16:
+            # the kernel forms these as the bf16 tile against the block's reference token times
+            # bf16 e^{Gam_ref}: two roundings
+            refs = np.repeat(Gam[sub // 2::sub], sub, axis=0)
+            with np.errstate(over="ignore"):
+                Kt = rnd(rnd(kc * np.exp(Gam - refs)) * rnd(np.exp(refs)))
+                Qt = rnd(rnd(qc * np.exp(Gam - refs)) * rnd(np.exp(refs)))
+        else:
+            Kt = kc * np.exp(Gam)
+            Qt = qc * np.exp(Gam)
         Kb = rnd(kc * np.exp(Gam[-1] - Gam))
         Sb = rnd(S)
         Y = vc - Kt @ Sb
