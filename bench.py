@@ -311,6 +311,35 @@ def run_ours(args):
     decode_ms = [e[1].elapsed_time(e[2]) for e in evs]
     total_ms, prefill_sum, decode_sum = max_over_ranks([total_ms, sum(prefill_ms), sum(decode_ms)], dev, world)
 
+    # ---- the same prefill writing the state every 512 tokens (prefix-cache boundaries), timed alone
+    states_line = None
+    if not args.no_states:
+        interval = 512
+        n_mid = P["T"] // interval
+        S_mid = torch.empty((P["B"], P["H"], n_mid, P["dk"], P["dv"]), dtype=torch.float32, device=dev)
+        for _ in range(2):
+            kda.kda_forward_chunked_states(q, k, v, g, beta, S0, interval=interval, o=o, S_T=ST, S_mid=S_mid,
+                                           stream=stream)
+        reps = max(3, min(args.steps, 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            kda.kda_forward_chunked_states(q, k, v, g, beta, S0, interval=interval, o=o, S_T=ST, S_mid=S_mid,
+                                           stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if kda.kda_get_device_status() != 0:
+            raise RuntimeError("device status after the state-emission run")
+        st_ms = e0.elapsed_time(e1) / reps
+        extra = P["B"] * P["H"] * n_mid * P["dk"] * P["dv"] * 4
+        st_bytes = prefill_alg_bytes(P["B"], P["T"], P["H"], P["dk"], P["dv"]) + extra
+        states_line = {"interval": interval, "states_per_head": n_mid, "launch_ms": st_ms,
+                       "tokens_per_s": P["B"] * P["T"] / (st_ms / 1e3), "extra_bytes": extra,
+                       "achieved_gbs": st_bytes / (st_ms / 1e3) / 1e9, "launches": reps,
+                       "timed": "separately, after the headline region (rank 0's own device)"}
+        del S_mid
+
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
     if args.no_e2e:
         e2e = None
@@ -356,6 +385,7 @@ def run_ours(args):
                    "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peak, "unit": "GB/s",
                                 "frac": dec_achieved / peak, "alg_bytes_per_launch": db_,
                                 "traffic": recorded_traffic("decode")}},
+        "state_emission": states_line,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": 2 * args.steps,
@@ -379,6 +409,7 @@ def main():
                     help="override the prefill workload (profiling small cases); the line is then not the headline")
     ap.add_argument("--decode-batch", type=int, default=None, help="override the decode batch (profiling)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--no-states", action="store_true", help="skip the state-emission (every 512 tokens) timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

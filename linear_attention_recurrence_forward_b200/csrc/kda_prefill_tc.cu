@@ -95,7 +95,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct TcParams {
     const __nv_bfloat16* beta;
     const float* S0;
-    __nv_bfloat16* o;
     float* ST;
     int* status;
     unsigned long long timeout_ns;  // limit of every mbarrier wait
@@ -194,7 +193,7 @@ __device__ __forceinline__ int tp_row(int r) { return r < 32 ? r : r + 32; }
 __global__ void __launch_bounds__(kThreads, 1)
 kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
-                      const TcParams p) {
+                      const __grid_constant__ CUtensorMap tm_o, const TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     // Align to 1024 B (the swizzle atoms need it) by offsetting the shared array itself, so the
     // compiler keeps every access in the shared state space.
@@ -226,7 +225,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         mbar_init(&bar_tpk, 1); mbar_init(&bar_drain_p, 1); mbar_init(&bar_drain_s, 1);
         fence_mbar_init();
         prefetch_tensormap(&tm_q); prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_g); prefetch_tensormap(&tm_v);
+        prefetch_tensormap(&tm_g); prefetch_tensormap(&tm_v); prefetch_tensormap(&tm_o);
     }
     if (warp == 0) {
         tmem_alloc(&tmem_base_s, TM_COLS);
@@ -583,7 +582,6 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         for (int chunk = 0; chunk < nchunks; ++chunk) {
             const uint32_t par = chunk & 1;
             const int t0 = chunk * kC;
-            const int nvalid = min(kC, T - t0);
             // ---- S1: MMA3 = [Qt0;Kt0;Qt1;Kt1] S once the prep group has the KQ tile (chunk 0 here;
             // later chunks issue it at the end of the previous chunk)
             if (stid == 0 && chunk == 0) {
@@ -672,9 +670,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc_fence_after_sync();
             ok = named_bar_and(kBarSerial, kSerialThreads, ok);
             if (!ok) break;
-            // ---- S4: the v tile is free: prefetch the next chunk's v.  S -> bf16 tile first (the next
-            // chunk's MMA3 waits on it), O read out of TMEM before MMA3 may overwrite it, stored after.
-            if (stid == 0 && chunk + 1 < nchunks) { load_v(chunk + 1); pending = chunk + 1; }
+            // ---- S4: S -> bf16 tile (the next chunk's MMA3 waits on it); O read out of TMEM before
+            // MMA3 may overwrite it and staged in the v tile (free now), which a TMA store writes out
             {
                 const int i = 32 * quarter + lane;
                 float sv[64];
@@ -690,35 +687,38 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         __stcs(reinterpret_cast<float4*>(dst + j), make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]));
                 }
             }
-            uint4 opk[8];   // O row segment, already rounded to bf16
             if ((quarter & 1) == 0) {
+                const int r = 32 * (quarter >> 1) + lane;   // token row of the chunk
                 float ov[64];
                 tmem_ld64(tlane + TM_C + 64 * colhalf, ov);   // warp-collective
 #pragma unroll
-                for (int j = 0; j < 8; ++j) opk[j] = pack8(ov + 8 * j);
+                for (int j = 0; j < 64; j += 8)
+                    *reinterpret_cast<uint4*>(sm + OFF_V + sw128_offset(r, 64 * colhalf + j, 8192)) = pack8(ov + j);
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
             named_bar_sync(kBarSerial, kSerialThreads);
-            if (stid == 0 && chunk + 1 < nchunks) {
-                ok = mbar_wait(&bar_kq, par ^ 1u, p.timeout_ns);
-                if (ok) {
-                    tc_fence_after_sync();
-                    issue_mma<8, false, 16384, true, 16384>(tbase + TM_C, sb + OFF_KQ, sb + OFF_SB, ID_KxMN, false);
-                    mma_commit(&bar_c);
-                }
-            }
-            if ((quarter & 1) == 0) {
-                const int r = 32 * (quarter >> 1) + lane;
-                if (r < nvalid) {
-                    uint4* orow = reinterpret_cast<uint4*>(p.o + (((size_t)b * T + t0 + r) * p.H + h) * kD + 64 * colhalf);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) orow[j] = opk[j];
+            if (stid == 0) {
+                // rows past T are clipped by the tensor map
+                tma_store_4d(&tm_o, sm + OFF_V, 0, h, t0, b);
+                tma_store_4d(&tm_o, sm + OFF_V + 8192, 64, h, t0, b);
+                bulk_commit_group();
+                if (chunk + 1 < nchunks) {
+                    bulk_wait_read_all();   // the staged O is read: the next v may land on it
+                    load_v(chunk + 1);
+                    pending = chunk + 1;
+                    ok = mbar_wait(&bar_kq, par ^ 1u, p.timeout_ns);
+                    if (ok) {
+                        tc_fence_after_sync();
+                        issue_mma<8, false, 16384, true, 16384>(tbase + TM_C, sb + OFF_KQ, sb + OFF_SB, ID_KxMN, false);
+                        mma_commit(&bar_c);
+                    }
                 }
             }
         }
         if (!ok && stid == 0) report_status(p.status, KDA_ERR_TIMEOUT);
         if (stid == 0) {
+            bulk_wait_all();
             mma_commit(&bar_drain_s);
             if (!mbar_wait(&bar_drain_s, 0, p.timeout_ns)) report_status(p.status, KDA_ERR_TIMEOUT);
             if (pending >= 0) (void)mbar_wait(&bar_v, (uint32_t)(pending & 1), p.timeout_ns);
@@ -790,13 +790,14 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
             attr_set[dev] = true;
         }
     }
-    CUtensorMap mq, mk, mg, mv;
+    CUtensorMap mq, mk, mg, mv, mo;
     if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
-        !make_map(&mg, a.g, a.B, a.T, a.H) || !make_map(&mv, a.v, a.B, a.T, a.H))
+        !make_map(&mg, a.g, a.B, a.T, a.H) || !make_map(&mv, a.v, a.B, a.T, a.H) ||
+        !make_map(&mo, a.o, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
-    TcParams prm{static_cast<const __nv_bfloat16*>(a.beta), a.S0, static_cast<__nv_bfloat16*>(a.o), a.ST,
+    TcParams prm{static_cast<const __nv_bfloat16*>(a.beta), a.S0, a.ST,
                  a.status, a.timeout_ns, a.skip_handoff, a.S_mid, a.interval, a.n_mid, a.B, a.T, a.H};
-    kda_prefill_tc_kernel<<<(unsigned)((size_t)a.B * a.H), kThreads, SMEM_DYN, s>>>(mq, mk, mg, mv, prm);
+    kda_prefill_tc_kernel<<<(unsigned)((size_t)a.B * a.H), kThreads, SMEM_DYN, s>>>(mq, mk, mg, mv, mo, prm);
     return cudaGetLastError();
 }
 
