@@ -162,6 +162,34 @@ __device__ __forceinline__ void load_b_frag(const float* blkT, int ld, int g, in
     b[0] = pack_bf16x2(v0.x, v0.y); b[1] = pack_bf16x2(v1.x, v1.y);
 }
 
+// 8x8 transpose of b16 pairs across the warp (thread i holds row i/4, columns 2(i%4) and 2(i%4)+1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+// A 16x16 fp32 tile held as two m16n8 accumulator tiles d[nt] (columns 8nt..8nt+7) ...
+// ... as the A operand (16x16, K = columns), rounded to bf16
+__device__ __forceinline__ void afrag_of_acc(const float d[2][4], uint32_t a[4]) {
+    a[0] = pack_bf16x2(d[0][0], d[0][1]); a[1] = pack_bf16x2(d[0][2], d[0][3]);
+    a[2] = pack_bf16x2(d[1][0], d[1][1]); a[3] = pack_bf16x2(d[1][2], d[1][3]);
+}
+// ... as the B operand (K = rows) of output columns 8nt..8nt+7, rounded to bf16
+__device__ __forceinline__ void bfrag_of_acc(const float d[2][4], int nt, uint32_t b[2]) {
+    b[0] = movmatrix_trans(pack_bf16x2(d[nt][0], d[nt][1]));
+    b[1] = movmatrix_trans(pack_bf16x2(d[nt][2], d[nt][3]));
+}
+// out = (acc ? out : 0) + X Y for 16x16 tiles held as accumulators (bf16 operands, fp32 sums)
+__device__ __forceinline__ void mm16_acc(float out[2][4], const uint32_t ax[4], const float y[2][4], bool acc) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        uint32_t b[2];
+        bfrag_of_acc(y, nt, b);
+        if (!acc) out[nt][0] = out[nt][1] = out[nt][2] = out[nt][3] = 0.f;
+        mma_16816(out[nt], ax, b);
+    }
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -456,36 +484,52 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             tc_fence_before_sync();  // the next chunk's MMA1 reuses these TMEM columns
             named_bar_sync(kBarPrep, kPrepThreads);
-            // diagonal 16x16 blocks of X = (I + A)^-1 by forward substitution, one lane per column:
-            // x_r = e_c[r] - sum_{l<r} A[r][l] x_l (the strictly upper entries of A are stored as 0)
-            if (warp < 2) {
-                const int blk = 2 * warp + (lane >> 4), c = lane & 15, o0 = 16 * blk;
-                float x[16];
+            // diagonal 16x16 blocks of X = (I + A)^-1, one warp per block: the strictly lower block N
+            // is nilpotent (N^16 = 0), so (I + N)^-1 = (I - N)(I + N^2)(I + N^4)(I + N^8), formed by
+            // warp-level tensor-core products (bf16 operands, fp32 sums) in four dependent rounds
+            if (warp < 4) {
+                const int o0 = 16 * warp, g4 = lane >> 2, t4 = lane & 3;
+                float nn[2][4], xm[2][4];  // N, then N^2, N^4, N^8; the running product
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const float* ar = AF + (o0 + r) * kLd + o0;
-                    float s0 = (r == c) ? 1.f : 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+                for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                    for (int l = 0; l < (r & ~3); l += 4) {
-                        const float4 a4 = *reinterpret_cast<const float4*>(ar + l);
-                        s0 = fmaf(-a4.x, x[l], s0); s1 = fmaf(-a4.y, x[l + 1], s1);
-                        s2 = fmaf(-a4.z, x[l + 2], s2); s3 = fmaf(-a4.w, x[l + 3], s3);
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int row = g4 + 8 * hr, col = 8 * nt + 2 * t4;
+                        const float2 v = *reinterpret_cast<const float2*>(AF + (o0 + row) * kLd + o0 + col);
+                        nn[nt][2 * hr] = v.x;
+                        nn[nt][2 * hr + 1] = v.y;
+                        xm[nt][2 * hr] = (row == col ? 1.f : 0.f) - v.x;
+                        xm[nt][2 * hr + 1] = (row == col + 1 ? 1.f : 0.f) - v.y;
                     }
 #pragma unroll
-                    for (int l = (r & ~3); l < r; ++l) s0 = fmaf(-ar[l], x[l], s0);
-                    x[r] = (s0 + s1) + (s2 + s3);
+                for (int round = 0; round < 3; ++round) {
+                    uint32_t an[4], ax[4];
+                    afrag_of_acc(nn, an);
+                    float sq[2][4];
+                    mm16_acc(sq, an, nn, false);        // N^(2^(round+1))
+                    afrag_of_acc(xm, ax);
+                    mm16_acc(xm, ax, sq, true);         // X <- X (I + N^(2^(round+1)))
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) nn[nt][e] = sq[nt][e];
                 }
+                // X, X^T (fp32, for the off-diagonal levels) and T = X Diag(beta) (bf16)
 #pragma unroll
-                for (int r = 0; r < 16; ++r) XF[(o0 + r) * kLd + o0 + c] = x[r];
+                for (int nt = 0; nt < 2; ++nt) {
+                    const int col = 8 * nt + 2 * t4;
+                    const float b0 = s_beta[o0 + col], b1 = s_beta[o0 + col + 1];
 #pragma unroll
-                for (int r = 0; r < 16; r += 4)
-                    *reinterpret_cast<float4*>(XT + (o0 + c) * kLd + o0 + r) = make_float4(x[r], x[r + 1], x[r + 2], x[r + 3]);
-                // T = X Diag(beta): this diagonal block's column c
-                const float bc = s_beta[o0 + c];
-#pragma unroll
-                for (int r = 0; r < 16; ++r)
-                    *reinterpret_cast<__nv_bfloat16*>(sm + OFF_T + sw128_offset(tp_row(o0 + r), o0 + c, 8192)) =
-                        __float2bfloat16_rn(x[r] * bc);
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int row = g4 + 8 * hr;
+                        const float x0 = xm[nt][2 * hr], x1 = xm[nt][2 * hr + 1];
+                        *reinterpret_cast<float2*>(XF + (o0 + row) * kLd + o0 + col) = make_float2(x0, x1);
+                        XT[(o0 + col) * kLd + o0 + row] = x0;
+                        XT[(o0 + col + 1) * kLd + o0 + row] = x1;
+                        *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(o0 + row), o0 + col, 8192)) =
+                            pack_bf16x2(x0 * b0, x1 * b1);
+                    }
+                }
             }
             named_bar_sync(kBarPrep, kPrepThreads);
             // X_RJ = -X_RR sum_{L=J}^{R-1} A_RL X_LJ by block distance d = R - J on warp-level bf16
