@@ -47,7 +47,37 @@ def _ftz(x):
     return np.where(np.abs(x) < 2.0 ** -126, 0.0, x)
 
 
-def chunk_head(q, k, v, g, beta, S0, C=64, sub=32, bf16=False, offdiag_ref="block_end"):
+def kernel_inverse(A, rnd):
+    """(I + A)^-1 for a strictly lower 64x64 A the way the tensor-core kernel forms it.
+
+    Diagonal 16x16 blocks: N = A_bb is nilpotent, (I + N)^-1 = (I - N)(I + N^2)(I + N^4)(I + N^8),
+    every product with operands rounded by `rnd` and exact sums.  Off-diagonal blocks by block
+    distance: X_RJ = -X_RR (sum_{L=J}^{R-1} A_RL X_LJ), operands rounded, the inner sum rounded
+    once more before the outer product.
+    """
+    n = A.shape[0]
+    nb = n // 16
+    X = np.zeros_like(A)
+    I16 = np.eye(16)
+    for b in range(nb):
+        s = slice(16 * b, 16 * b + 16)
+        N = A[s, s]
+        P = I16 - N
+        Np = N
+        for _ in range(3):
+            Np = rnd(Np) @ rnd(Np)
+            P = P + rnd(P) @ rnd(Np)
+        X[s, s] = P
+    for d in range(1, nb):
+        for J in range(nb - d):
+            R = J + d
+            rs, js = slice(16 * R, 16 * R + 16), slice(16 * J, 16 * J + 16)
+            W = sum(rnd(A[rs, 16 * L:16 * L + 16]) @ rnd(X[16 * L:16 * L + 16, js]) for L in range(J, R))
+            X[rs, js] = -(rnd(X[rs, rs]) @ rnd(W))
+    return X
+
+
+def chunk_head(q, k, v, g, beta, S0, C=64, sub=32, bf16=False, offdiag_ref="block_end", solve="exact"):
     """One head. q,k,g [T,dk]; v [T,dv]; beta [T]; S0 [dk,dv]. Returns (o [T,dv], S_T).
 
     offdiag_ref: reference token of an off-diagonal block pair (R > J).  "block_end" factors at
@@ -56,6 +86,9 @@ def chunk_head(q, k, v, g, beta, S0, C=64, sub=32, bf16=False, offdiag_ref="bloc
     below the fp32 normal range to zero: this is what the tensor-core kernel does for C = 64,
     sub = 32 (one product for the whole block row).  The kernel builds those column factors from
     in-range pieces, so it flushes no more than this model does.
+
+    solve: "exact" solves (I + A) T = Diag(beta) in fp64; "kernel" forms (I + A)^-1 as the tensor-core
+    kernel does (kernel_inverse, with the bf16 rounding when bf16=True; needs C = 64).
     """
     T, dk = q.shape
     dv = v.shape[1]
@@ -93,7 +126,10 @@ def chunk_head(q, k, v, g, beta, S0, C=64, sub=32, bf16=False, offdiag_ref="bloc
         with np.errstate(invalid="ignore", over="ignore"):
             P = np.where(np.tril(np.ones((C, C), bool)), P, 0.0)
             A = np.where(np.tril(np.ones((C, C), bool), -1), A, 0.0) * bc[:, None]
-        Tm = np.linalg.solve(np.eye(C) + A, np.diag(bc))
+        if solve == "kernel":
+            Tm = kernel_inverse(A, rnd) * bc[None, :]
+        else:
+            Tm = np.linalg.solve(np.eye(C) + A, np.diag(bc))
         if bf16:
             # the kernel forms these as the bf16 tile against the block's reference token times
             # bf16 e^{Gam_ref}: two roundings
@@ -115,7 +151,7 @@ def chunk_head(q, k, v, g, beta, S0, C=64, sub=32, bf16=False, offdiag_ref="bloc
     return o, S
 
 
-def chunk_forward(q, k, v, g, beta, S0=None, C=64, sub=32, bf16=False, offdiag_ref="block_end"):
+def chunk_forward(q, k, v, g, beta, S0=None, C=64, sub=32, bf16=False, offdiag_ref="block_end", solve="exact"):
     """[B,T,H,*] fp64 arrays -> (o [B,T,H,dv], S_T [B,H,dk,dv])."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -126,5 +162,5 @@ def chunk_forward(q, k, v, g, beta, S0=None, C=64, sub=32, bf16=False, offdiag_r
             s0 = np.zeros((dk, dv)) if S0 is None else S0[b, h]
             o[b, :, h], ST[b, h] = chunk_head(q[b, :, h], k[b, :, h], v[b, :, h], g[b, :, h],
                                               beta[b, :, h], s0, C=C, sub=sub, bf16=bf16,
-                                              offdiag_ref=offdiag_ref)
+                                              offdiag_ref=offdiag_ref, solve=solve)
     return o, ST

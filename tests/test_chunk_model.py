@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 
 import oracle
-from chunk_model import chunk_forward
+from chunk_model import kernel_inverse, chunk_forward
 from helpers import max_rel_err, random_problem
 
 
@@ -42,7 +42,8 @@ def test_bf16_operands_stay_inside_tolerance(zg_mean):
     q, k, v, g, beta, S0 = random_problem(rng, 1, 320, 1, 64, 64)
     g = -5.0 / (1.0 + np.exp(-(rng.standard_normal(g.shape) + zg_mean)))
     o_ref, ST_ref = oracle.forward(q, k, v, g, beta, S0, nthreads=2)
-    o, ST = chunk_forward(q, k, v, g, beta, S0, C=64, sub=32, bf16=True)
+    o, ST = chunk_forward(q, k, v, g, beta, S0, C=64, sub=32, bf16=True, offdiag_ref="row_middle",
+                          solve="kernel")
     # half the 2e-2 bf16 tolerance, before the final bf16 rounding of o
     assert max_rel_err(o, o_ref) < 1e-2, max_rel_err(o, o_ref)
     assert max_rel_err(ST, ST_ref) < 1e-2, max_rel_err(ST, ST_ref)
@@ -72,3 +73,15 @@ def test_kernel_factorisation_stays_close_to_oracle(pattern):
     o, ST = chunk_forward(q, k, v, g, beta, S0, C=64, sub=32, offdiag_ref="row_middle")
     assert max_rel_err(o, o_ref) < 1e-3, max_rel_err(o, o_ref)
     assert max_rel_err(ST, ST_ref) < 1e-3, max_rel_err(ST, ST_ref)
+
+
+def test_kernel_inverse_is_the_inverse_in_exact_arithmetic():
+    """The doubling and block-distance recurrences give (I + A)^-1 exactly (no rounding)."""
+    rng = np.random.default_rng(12)
+    A = np.tril(rng.standard_normal((64, 64)) * 0.3, -1)
+    X = kernel_inverse(A, lambda x: x)
+    assert np.max(np.abs(X - np.linalg.inv(np.eye(64) + A))) < 1e-10
+    # a plausible slip (one doubling round fewer) is caught
+    N = A[:16, :16]
+    short = (np.eye(16) - N) @ (np.eye(16) + N @ N) @ (np.eye(16) + np.linalg.matrix_power(N, 4))
+    assert np.max(np.abs(short - np.linalg.inv(np.eye(16) + N))) > 1e-6
