@@ -417,14 +417,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             fence_proxy_async_smem();
             tc_fence_before_sync();
             named_bar_sync(kBarPrep, kPrepThreads);
-            if (ptid == kIssuer) {
-                tc_fence_after_sync();
-                if (!(p.skip_handoff && chunk == 0)) mbar_arrive(&bar_kq);  // KQ of this chunk is ready for MMA3
-                issue_mma<8, false, 16384, false, 12288>(tbase + TM_P, sb + OFF_A1, sb + OFF_BB, ID_MMA1, false);
-                mma_commit(&bar_ap);
-                // raw q,k,g are consumed (Gam was read before the barrier): prefetch the next chunk
-                if (chunk + 1 < nchunks) { load_qkg(chunk + 1); pending = chunk + 1; }
-            }
+            // A1, BB and KQ of this chunk are ready and its raw q, k, g consumed: the recurrence group's
+            // leader issues MMA1, MMA3 and the next chunk's loads
+            if (ptid == kIssuer && !(p.skip_handoff && chunk == 0)) mbar_arrive(&bar_kq);
             // ---- P4: Kb tile, P and A from TMEM, triangular solve, T tile
             if (chunk > 0) ok = mbar_wait(&bar_os, ppar, p.timeout_ns);  // T, P, Kb released
             if (ok) {
@@ -596,6 +591,18 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // ====================================================================== serial group
         const int stid = tid - kPrepThreads;                // 0..255
         int pending = -1;                                   // chunk whose v load is in flight
+        int pending_qkg = -1;                               // last chunk whose q,k,g loads this leader issued
+        // Once the prep group has published chunk c's operand tiles (bar_kq): MMA1 (its A and P
+        // products, on the prep group's path, so first), MMA3 = [Qt0;Kt0;Qt1;Kt1] S, and the raw
+        // q, k, g of chunk c+1 into the buffers the prep group has finished reading.
+        auto issue_for_chunk = [&](int c) {
+            tc_fence_after_sync();
+            issue_mma<8, false, 16384, false, 12288>(tbase + TM_P, sb + OFF_A1, sb + OFF_BB, ID_MMA1, false);
+            mma_commit(&bar_ap);
+            issue_mma<8, false, 16384, true, 16384>(tbase + TM_C, sb + OFF_KQ, sb + OFF_SB, ID_KxMN, false);
+            mma_commit(&bar_c);
+            if (c + 1 < nchunks) { load_qkg(c + 1); pending_qkg = c + 1; }
+        };
         // initial state: fp32 into TMEM, bf16 copy into the MN-major S tile
         {
             const int i = 32 * quarter + lane;
@@ -626,15 +633,11 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         for (int chunk = 0; chunk < nchunks; ++chunk) {
             const uint32_t par = chunk & 1;
             const int t0 = chunk * kC;
-            // ---- S1: MMA3 = [Qt0;Kt0;Qt1;Kt1] S once the prep group has the KQ tile (chunk 0 here;
-            // later chunks issue it at the end of the previous chunk)
+            // ---- S1: MMA1 and MMA3 once the prep group has the operand tiles (chunk 0 here; later
+            // chunks issue them at the end of the previous chunk)
             if (stid == 0 && chunk == 0) {
                 ok = mbar_wait(&bar_kq, par, p.timeout_ns);
-                if (ok) {
-                    tc_fence_after_sync();
-                    issue_mma<8, false, 16384, true, 16384>(tbase + TM_C, sb + OFF_KQ, sb + OFF_SB, ID_KxMN, false);
-                    mma_commit(&bar_c);
-                }
+                if (ok) issue_for_chunk(0);
             }
             // Y = V - Kt S (Kt rows sit in lanes 32-63 and 96-127), in place over v
             if (ok) ok = mbar_wait(&bar_c, par, p.timeout_ns);
@@ -752,11 +755,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     load_v(chunk + 1);
                     pending = chunk + 1;
                     ok = mbar_wait(&bar_kq, par ^ 1u, p.timeout_ns);
-                    if (ok) {
-                        tc_fence_after_sync();
-                        issue_mma<8, false, 16384, true, 16384>(tbase + TM_C, sb + OFF_KQ, sb + OFF_SB, ID_KxMN, false);
-                        mma_commit(&bar_c);
-                    }
+                    if (ok) issue_for_chunk(chunk + 1);
                 }
             }
         }
@@ -766,6 +765,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mma_commit(&bar_drain_s);
             if (!mbar_wait(&bar_drain_s, 0, p.timeout_ns)) report_status(p.status, KDA_ERR_TIMEOUT);
             if (pending >= 0) (void)mbar_wait(&bar_v, (uint32_t)(pending & 1), p.timeout_ns);
+            if (pending_qkg >= 0) (void)mbar_wait(&bar_qkg, (uint32_t)(pending_qkg & 1), p.timeout_ns);
         }
         named_bar_sync(kBarSerial, kSerialThreads);
         tc_fence_after_sync();
