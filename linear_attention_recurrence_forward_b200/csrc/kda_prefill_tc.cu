@@ -311,12 +311,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // ---- P1: beta; this chunk's q, k, g
             if (ptid < kC) s_beta[ptid] = __uint_as_float((uint32_t)beta_next << 16);
             if (chunk + 1 < nchunks) beta_next = fetch_beta(chunk + 1);
-            if (ptid == kIssuer) {
-                ok = mbar_wait(&bar_qkg, par, p.timeout_ns);
-                if (ok) pending = -1;
-            }
-            ok = named_bar_and(kBarPrep, kPrepThreads, ok);
-            if (!ok) break;
+            ok = mbar_wait(&bar_qkg, par, p.timeout_ns);   // every thread: its own view of the TMA data
+            if (ok && ptid == kIssuer) pending = -1;
             // ---- P2: Gam = in-chunk prefix sum of g in fp32: the running sum over this quarter,
             // then the totals of the quarters before it
             float gam[16][2];
@@ -332,7 +328,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
                 *reinterpret_cast<float2*>(&s_qsum[tq][ch0]) = make_float2(a0, a1);
             }
-            named_bar_sync(kBarPrep, kPrepThreads);
+            ok = named_bar_and(kBarPrep, kPrepThreads, ok);
+            if (!ok) break;
             {
                 float c0s = 0.f, c1s = 0.f;
 #pragma unroll 1
@@ -428,10 +425,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     *reinterpret_cast<uint32_t*>(sm + OFF_KBAR + sw128_offset(16 * tq + i, ch0, 8192)) = kb[i];
             }
             if (ok) ok = mbar_wait(&bar_ap, par, p.timeout_ns);
+            ok = __all_sync(0xffffffffu, ok);   // warp-uniform: the TMEM loads below are warp-collective
             tc_fence_after_sync();
-            ok = named_bar_and(kBarPrep, kPrepThreads, ok);
-            if (!ok) break;
-            {
+            if (ok) {
                 // TMEM lane L of MMA1: quarter 0 Qt0 rows, 1 Kt0 rows, 2 Qt1 rows, 3 Kt1 rows.
                 // Columns of a row r: j < 32 from cols 0..31 (block 0) or 64..95 (block 1 rows);
                 // j >= 32 zero (block 0) or cols 32..63 (block 1).  colhalf picks j < 32 / j >= 32.
@@ -478,7 +474,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
             }
             tc_fence_before_sync();  // the next chunk's MMA1 reuses these TMEM columns
-            named_bar_sync(kBarPrep, kPrepThreads);
+            ok = named_bar_and(kBarPrep, kPrepThreads, ok);
+            if (!ok) break;
             // diagonal 16x16 blocks of X = (I + A)^-1, one warp per block: the strictly lower block N
             // is nilpotent (N^16 = 0), so (I + N)^-1 = (I - N)(I + N^2)(I + N^4)(I + N^8), formed by
             // warp-level tensor-core products (bf16 operands, fp32 sums) in four dependent rounds
