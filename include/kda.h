@@ -145,6 +145,27 @@ KDA_API int kda_decode_step(const void* q, const void* k, const void* v, const v
                     int dtype, struct CUstream_st* stream);
 
 /*
+ * kda_state_compose -- apply a segment's state map: S_out = M S_in + N for `count` heads (fp32).
+ *
+ * Over a segment of tokens the recurrence is affine in its initial state: S_end = M S_start + N,
+ * with M = prod_t (I - beta_t k_t k_t^T) Diag(exp g_t) and N the final state from a zero start.
+ * Splitting a long sequence over devices then only needs this fixed-size pair exchanged
+ * (KDA context parallelism: channel post on the K3 report (t.iss.one), infrastructure
+ * paragraph).  A segment's pair comes from two kda_forward_chunked calls: N with S0 = NULL,
+ * M as S_T with v = 0 (dv = dk) and S0 = the identity.
+ *
+ *   M      : [count, dk, dk] fp32
+ *   S_in   : [count, dk, dv] fp32
+ *   N      : [count, dk, dv] fp32, or NULL for zero
+ *   S_out  : [count, dk, dv] fp32 output; may be S_in or N itself (in place), must not
+ *            overlap M or partially overlap S_in / N
+ *
+ * dk, dv in {64, 128}.  Returns KDA_OK or a negative kda_status (nothing enqueued on error).
+ */
+KDA_API int kda_state_compose(const float* M, const float* S_in, const float* N, float* S_out, int count,
+                              int dk, int dv, struct CUstream_st* stream);
+
+/*
  * kda_get_device_status -- synchronise `stream`, then return and clear the status word
  * of the current device: KDA_OK, KDA_ERR_TIMEOUT (a kernel's bounded wait gave up; its
  * outputs are then undefined), or KDA_ERR_CUDA if the synchronisation itself failed.

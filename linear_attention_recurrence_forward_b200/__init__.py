@@ -25,6 +25,7 @@ __all__ = [
     "kda_forward_chunked",
     "kda_forward_chunked_states",
     "kda_decode_step",
+    "kda_state_compose",
     "kda_get_device_status",
     "kda_status_string",
     "kda_debug_set_wait_fault",
@@ -74,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.kda_forward_chunked_impl.restype = I
         L.kda_forward_chunked_states.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]
         L.kda_forward_chunked_states.restype = I
+        L.kda_state_compose.argtypes = [P, P, P, P, I, I, I, P]
+        L.kda_state_compose.restype = I
         L.kda_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P]
         L.kda_decode_step.restype = I
         L.kda_get_device_status.argtypes = [P]
@@ -209,6 +212,32 @@ def kda_decode_step(q, k, v, g, beta, S, *, o=None, stream=None):
     if rc != 0:
         raise KdaError("kda_decode_step", rc)
     return o
+
+
+def kda_state_compose(M, S, N=None, *, out=None, stream=None):
+    """out = M @ S + N per head: M [..., dk, dk], S and N [..., dk, dv] fp32 CUDA tensors (N may be None).
+
+    out may be S or N itself.  The leading dimensions are flattened into heads.
+    """
+    dk, dv = S.shape[-2], S.shape[-1]
+    lead = tuple(S.shape[:-2])
+    dev = S.device
+    _check(M, "M", lead + (dk, dk), torch.float32, dev)
+    if N is not None:
+        _check(N, "N", lead + (dk, dv), torch.float32, dev)
+    _check(S, "S", lead + (dk, dv), torch.float32, dev)
+    if out is None:
+        out = torch.empty_like(S)
+    else:
+        _check(out, "out", lead + (dk, dv), torch.float32, dev)
+    count = 1
+    for x in lead:
+        count *= x
+    with torch.cuda.device(dev):
+        rc = lib().kda_state_compose(_ptr(M), _ptr(S), _ptr(N), _ptr(out), count, dk, dv, _stream_handle(stream))
+    if rc != 0:
+        raise KdaError("kda_state_compose", rc)
+    return out
 
 
 def kda_get_device_status(stream=None, device=None) -> int:

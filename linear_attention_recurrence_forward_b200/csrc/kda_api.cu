@@ -196,6 +196,25 @@ int kda_decode_step(const void* q, const void* k, const void* v, const void* g, 
     return kda::launch_decode(a, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+int kda_state_compose(const float* M, const float* S_in, const float* N, float* S_out, int count, int dk,
+                      int dv, struct CUstream_st* stream) {
+    if (count <= 0) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (!M || !S_in || !S_out) return KDA_ERR_INVALID_ARG;
+    if ((double)count * dk * (dk > dv ? dk : dv) > 9.0e15) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {M, S_in, N, S_out};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    const size_t sbytes = (size_t)count * dk * dv * sizeof(float);
+    const Range rm = range_of(M, (size_t)count * dk * dk * sizeof(float));
+    const Range ro = range_of(S_out, sbytes);
+    if (overlaps(rm, ro)) return KDA_ERR_INVALID_ARG;
+    // S_out may be S_in or N exactly; any other overlap is not allowed
+    if (S_out != S_in && overlaps(ro, range_of(S_in, sbytes))) return KDA_ERR_INVALID_ARG;
+    if (N && S_out != N && overlaps(ro, range_of(N, sbytes))) return KDA_ERR_INVALID_ARG;
+    return kda::launch_state_compose(M, S_in, N, S_out, count, dk, dv, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 int kda_get_device_status(struct CUstream_st* stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
     int* addr = status_word_for_current_device();

@@ -47,6 +47,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 bool prefill_tc_supports(const PrefillArgs& a);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_state_compose(const float* M, const float* S, const float* N, float* out, int count, int dk,
+                                 int dv, cudaStream_t s);
 
 // Element loads/stores for the two input dtypes.
 __device__ __forceinline__ float load_elem(const float* p, size_t i) { return p[i]; }

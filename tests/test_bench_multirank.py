@@ -37,7 +37,7 @@ def _rank_main(rank, world, port, out):
 
 
 def test_max_over_ranks_and_weak_scaling_with_two_gloo_ranks():
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     port = 29500 + (os.getpid() % 1000)
     mp.start_processes(_rank_main, args=(2, port, out), nprocs=2, join=True, start_method="spawn")
