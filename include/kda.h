@@ -145,6 +145,48 @@ KDA_API int kda_decode_step(const void* q, const void* k, const void* v, const v
                     int dtype, struct CUstream_st* stream);
 
 /*
+ * kda_forward_varlen -- prefill over packed sequences of different lengths (continuous batching).
+ *
+ * N sequences stored back to back along the token axis (the layout a paged serving engine
+ * batches prefills in; podcast show-notes (scripod.com), outline item 5.3.1, and the channel
+ * post on the K3 report (t.iss.one), online-inference paragraph: one paged pool for the KDA
+ * states):
+ *
+ *   q, k, g    : [T_total, H, dk]   dtype
+ *   v          : [T_total, H, dv]   dtype
+ *   beta       : [T_total, H]       dtype
+ *   cu_seqlens : [N + 1] int32 DEVICE array: sequence n is tokens cu_seqlens[n] .. cu_seqlens[n+1]-1,
+ *                0 <= cu_seqlens[n] <= cu_seqlens[n+1] <= T_total.  The kernels check it: a sequence
+ *                whose range is invalid is processed as empty (S_T = S0) and the device status word
+ *                is set to KDA_ERR_INVALID_ARG.  o rows of tokens outside every range are not written.
+ *   S0, S_T    : [N, H, dk, dv] fp32, S0 may be NULL (zeros), S_T may be NULL or alias S0
+ *   o          : [T_total, H, dv]   dtype
+ *   impl       : kda_impl.
+ *
+ * Every sequence gives exactly what kda_forward_chunked gives for it alone.  Returns KDA_OK
+ * or a negative kda_status (nothing enqueued on error).
+ */
+KDA_API int kda_forward_varlen(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                               const int* cu_seqlens, const float* S0, void* o, float* S_T, int N,
+                               int T_total, int H, int dk, int dv, int dtype, int impl,
+                               struct CUstream_st* stream);
+
+/*
+ * kda_decode_step_paged -- kda_decode_step with the states in a pool indexed per sequence.
+ *
+ *   S_pool : [n_slots, H, dk, dv] fp32, read and written in place
+ *   slots  : [B] int32 DEVICE array: sequence b uses S_pool[slots[b]]; slots[b] < 0 skips sequence
+ *            b (nothing read or written, o[b] untouched).  Active slots must be distinct.  A slot
+ *            >= n_slots is skipped and sets the device status word to KDA_ERR_INVALID_ARG.
+ *   q, k, g, v, beta, o : as kda_decode_step (per sequence b).
+ *
+ * Returns KDA_OK or a negative kda_status (nothing enqueued on error).
+ */
+KDA_API int kda_decode_step_paged(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                                  float* S_pool, int n_slots, const int* slots, void* o, int B, int H,
+                                  int dk, int dv, int dtype, struct CUstream_st* stream);
+
+/*
  * kda_state_compose -- apply a segment's state map: S_out = M S_in + N for `count` heads (fp32).
  *
  * Over a segment of tokens the recurrence is affine in its initial state: S_end = M S_start + N,
@@ -168,7 +210,9 @@ KDA_API int kda_state_compose(const float* M, const float* S_in, const float* N,
 /*
  * kda_get_device_status -- synchronise `stream`, then return and clear the status word
  * of the current device: KDA_OK, KDA_ERR_TIMEOUT (a kernel's bounded wait gave up; its
- * outputs are then undefined), or KDA_ERR_CUDA if the synchronisation itself failed.
+ * outputs are then undefined), KDA_ERR_INVALID_ARG (a kernel found an out-of-range device
+ * index: a sequence offset or a state slot), or KDA_ERR_CUDA if the synchronisation itself
+ * failed.
  */
 KDA_API int kda_get_device_status(struct CUstream_st* stream);
 

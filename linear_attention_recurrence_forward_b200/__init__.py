@@ -25,6 +25,8 @@ __all__ = [
     "kda_forward_chunked",
     "kda_forward_chunked_states",
     "kda_decode_step",
+    "kda_forward_varlen",
+    "kda_decode_step_paged",
     "kda_state_compose",
     "kda_get_device_status",
     "kda_status_string",
@@ -77,6 +79,10 @@ def lib() -> ctypes.CDLL:
         L.kda_forward_chunked_states.restype = I
         L.kda_state_compose.argtypes = [P, P, P, P, I, I, I, P]
         L.kda_state_compose.restype = I
+        L.kda_forward_varlen.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P]
+        L.kda_forward_varlen.restype = I
+        L.kda_decode_step_paged.argtypes = [P, P, P, P, P, P, I, P, P, I, I, I, I, I, P]
+        L.kda_decode_step_paged.restype = I
         L.kda_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P]
         L.kda_decode_step.restype = I
         L.kda_get_device_status.argtypes = [P]
@@ -211,6 +217,67 @@ def kda_decode_step(q, k, v, g, beta, S, *, o=None, stream=None):
                                    B, H, dk, dv, DTYPE[dt], _stream_handle(stream))
     if rc != 0:
         raise KdaError("kda_decode_step", rc)
+    return o
+
+
+def kda_forward_varlen(q, k, v, g, beta, cu_seqlens, S0=None, *, o=None, S_T=None, return_state: bool = True,
+                       impl: str = "auto", stream=None):
+    """Prefill over packed sequences: q, k, g [T_total, H, dk]; v [T_total, H, dv]; beta [T_total, H];
+    cu_seqlens int32 [N + 1] on the device (sequence n = tokens cu_seqlens[n] .. cu_seqlens[n+1]-1).
+    States [N, H, dk, dv] fp32.  Returns (o [T_total, H, dv], S_T or None).
+    """
+    T_total, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.shape[0] - 1
+    dev, dt = q.device, q.dtype
+    if dt not in DTYPE:
+        raise ValueError(f"unsupported dtype {dt}")
+    for name, t, shape in (("q", q, (T_total, H, dk)), ("k", k, (T_total, H, dk)), ("v", v, (T_total, H, dv)),
+                           ("g", g, (T_total, H, dk)), ("beta", beta, (T_total, H))):
+        _check(t, name, shape, dt, dev)
+    _check(cu_seqlens, "cu_seqlens", (N + 1,), torch.int32, dev)
+    if S0 is not None:
+        _check(S0, "S0", (N, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty((T_total, H, dv), dtype=dt, device=dev)
+    else:
+        _check(o, "o", (T_total, H, dv), dt, dev)
+    if S_T is None and return_state:
+        S_T = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    elif S_T is not None:
+        _check(S_T, "S_T", (N, H, dk, dv), torch.float32, dev)
+    with torch.cuda.device(dev):
+        rc = lib().kda_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), _ptr(S0),
+                                      _ptr(o), _ptr(S_T), N, T_total, H, dk, dv, DTYPE[dt], IMPL[impl],
+                                      _stream_handle(stream))
+    if rc != 0:
+        raise KdaError("kda_forward_varlen", rc)
+    return o, S_T
+
+
+def kda_decode_step_paged(q, k, v, g, beta, S_pool, slots, *, o=None, stream=None):
+    """One token per sequence with the states in a pool: S_pool [n_slots, H, dk, dv] fp32 (updated in
+    place), slots int32 [B] on the device (sequence b uses S_pool[slots[b]]; negative = skip)."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    if dt not in DTYPE:
+        raise ValueError(f"unsupported dtype {dt}")
+    for name, t, shape in (("q", q, (B, H, dk)), ("k", k, (B, H, dk)), ("v", v, (B, H, dv)),
+                           ("g", g, (B, H, dk)), ("beta", beta, (B, H))):
+        _check(t, name, shape, dt, dev)
+    n_slots = S_pool.shape[0]
+    _check(S_pool, "S_pool", (n_slots, H, dk, dv), torch.float32, dev)
+    _check(slots, "slots", (B,), torch.int32, dev)
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=dt, device=dev)
+    else:
+        _check(o, "o", (B, H, dv), dt, dev)
+    with torch.cuda.device(dev):
+        rc = lib().kda_decode_step_paged(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S_pool), n_slots,
+                                         _ptr(slots), _ptr(o), B, H, dk, dv, DTYPE[dt], _stream_handle(stream))
+    if rc != 0:
+        raise KdaError("kda_decode_step_paged", rc)
     return o
 
 

@@ -52,7 +52,8 @@ size_t elem_size(int dtype) { return dtype == KDA_DTYPE_BF16 ? 2 : 4; }
 
 int validate_prefill(const void* q, const void* k, const void* v, const void* g, const void* beta,
                      const float* S0, const void* o, const float* ST, int B, int T, int H, int dk,
-                     int dv, int dtype) {
+                     int dv, int dtype, int n_states = -1) {
+    if (n_states < 0) n_states = B;   // states [n_states, H, dk, dv]
     if (B <= 0 || H <= 0 || T < 0) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_FP32) return KDA_ERR_UNSUPPORTED;
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
@@ -72,7 +73,7 @@ int validate_prefill(const void* q, const void* k, const void* v, const void* g,
                              range_of(beta, n_tok * es)};
         for (const Range& r : ins)
             if (overlaps(ro, r)) return KDA_ERR_INVALID_ARG;
-        const size_t sbytes = (size_t)B * H * dk * dv * sizeof(float);
+        const size_t sbytes = (size_t)n_states * H * dk * dv * sizeof(float);
         if (S0 && overlaps(ro, range_of(S0, sbytes))) return KDA_ERR_INVALID_ARG;
         if (ST) {
             const Range rs = range_of(ST, sbytes);
@@ -82,7 +83,7 @@ int validate_prefill(const void* q, const void* k, const void* v, const void* g,
         }
     }
     if (S0 && ST && S0 != ST) {
-        const size_t sbytes = (size_t)B * H * dk * dv * sizeof(float);
+        const size_t sbytes = (size_t)n_states * H * dk * dv * sizeof(float);
         if (overlaps(range_of(S0, sbytes), range_of(ST, sbytes))) return KDA_ERR_INVALID_ARG;
     }
     return KDA_OK;
@@ -114,11 +115,21 @@ int validate_states(const void* q, const void* k, const void* v, const void* g, 
 
 int forward_impl(const void* q, const void* k, const void* v, const void* g, const void* beta,
                  const float* S0, void* o, float* ST, int B, int T, int H, int dk, int dv, int dtype,
-                 int impl, cudaStream_t stream, float* S_mid = nullptr, int interval = 0) {
+                 int impl, cudaStream_t stream, float* S_mid = nullptr, int interval = 0,
+                 const int* cu_seqlens = nullptr) {
     if (impl != KDA_IMPL_AUTO && impl != KDA_IMPL_TCGEN05 && impl != KDA_IMPL_SIMT)
         return KDA_ERR_INVALID_ARG;
-    int rc = validate_prefill(q, k, v, g, beta, S0, o, ST, B, T, H, dk, dv, dtype);
+    // packed sequences: the activations are one batch entry of T tokens, the states B entries
+    int rc = cu_seqlens ? validate_prefill(q, k, v, g, beta, S0, o, ST, 1, T, H, dk, dv, dtype, B)
+                        : validate_prefill(q, k, v, g, beta, S0, o, ST, B, T, H, dk, dv, dtype);
     if (rc != KDA_OK) return rc;
+    if (cu_seqlens) {
+        if (!aligned16(cu_seqlens)) return KDA_ERR_MISALIGNED;
+        const Range rc_ = range_of(cu_seqlens, (size_t)(B + 1) * sizeof(int));
+        const size_t es = elem_size(dtype);
+        if (T > 0 && overlaps(rc_, range_of(o, (size_t)T * H * dv * es))) return KDA_ERR_INVALID_ARG;
+        if (ST && overlaps(rc_, range_of(ST, (size_t)B * H * dk * dv * sizeof(float)))) return KDA_ERR_INVALID_ARG;
+    }
     int n_mid = 0;
     if (interval != 0 || S_mid) {
         rc = validate_states(q, k, v, g, beta, S0, o, ST, S_mid, interval, B, T, H, dk, dv, dtype, &n_mid);
@@ -126,7 +137,7 @@ int forward_impl(const void* q, const void* k, const void* v, const void* g, con
     }
     kda::PrefillArgs a{q, k, v, g, beta, S0, o, ST, B, T, H, dk, dv, dtype, nullptr,
                        g_timeout_ns.load(), g_skip_handoff.load(), n_mid > 0 ? S_mid : nullptr,
-                       interval, n_mid};
+                       interval, n_mid, cu_seqlens};
     const bool tc_ok = kda::prefill_tc_supports(a);
     if (impl == KDA_IMPL_TCGEN05 && !tc_ok) return KDA_ERR_UNSUPPORTED;
     if (T == 0) {
@@ -144,6 +155,38 @@ int forward_impl(const void* q, const void* k, const void* v, const void* g, con
     if (impl == KDA_IMPL_SIMT || (impl == KDA_IMPL_AUTO && !tc_ok)) e = kda::launch_prefill_simt(a, stream);
     else e = kda::launch_prefill_tc(a, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int decode_impl(const void* q, const void* k, const void* v, const void* g, const void* beta, float* S,
+                int n_slots, const int* slots, void* o, int B, int H, int dk, int dv, int dtype,
+                cudaStream_t stream) {
+    if (B <= 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_FP32) return KDA_ERR_UNSUPPORTED;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !g || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
+    if ((double)B * (double)H > 2.0e9) return KDA_ERR_INVALID_ARG;
+    if (slots && (n_slots <= 0 || (double)n_slots * (double)H > 2.0e9)) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, g, beta, S, o, slots ? (const void*)slots : (const void*)q};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+    const size_t es = elem_size(dtype);
+    const size_t n = (size_t)B * H;
+    const size_t n_state = slots ? (size_t)n_slots * H : n;
+    const Range rs = range_of(S, n_state * dk * dv * sizeof(float));
+    const Range ro = range_of(o, n * dv * es);
+    const Range ins[] = {range_of(q, n * dk * es), range_of(k, n * dk * es), range_of(v, n * dv * es),
+                         range_of(g, n * dk * es), range_of(beta, n * es)};
+    if (overlaps(rs, ro)) return KDA_ERR_INVALID_ARG;
+    for (const Range& r : ins)
+        if (overlaps(rs, r) || overlaps(ro, r)) return KDA_ERR_INVALID_ARG;
+    if (slots) {
+        const Range rt = range_of(slots, (size_t)B * sizeof(int));
+        if (overlaps(rt, rs) || overlaps(rt, ro)) return KDA_ERR_INVALID_ARG;
+    }
+    kda::DecodeArgs a{q, k, v, g, beta, S, o, B, H, dk, dv, dtype, status_word_for_current_device(), slots,
+                      n_slots};
+    if (!a.status) return KDA_ERR_CUDA;
+    return kda::launch_decode(a, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 }  // namespace
@@ -171,29 +214,25 @@ int kda_forward_chunked_states(const void* q, const void* k, const void* v, cons
                         interval);
 }
 
+int kda_forward_varlen(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                       const int* cu_seqlens, const float* S0, void* o, float* S_T, int N, int T_total,
+                       int H, int dk, int dv, int dtype, int impl, struct CUstream_st* stream) {
+    if (N <= 0 || !cu_seqlens) return KDA_ERR_INVALID_ARG;
+    return forward_impl(q, k, v, g, beta, S0, o, S_T, N, T_total, H, dk, dv, dtype, impl, stream, nullptr, 0,
+                        cu_seqlens);
+}
+
 int kda_decode_step(const void* q, const void* k, const void* v, const void* g, const void* beta,
                     float* S, void* o, int B, int H, int dk, int dv, int dtype,
                     struct CUstream_st* stream) {
-    if (B <= 0 || H <= 0) return KDA_ERR_INVALID_ARG;
-    if (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_FP32) return KDA_ERR_UNSUPPORTED;
-    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
-    if (!q || !k || !v || !g || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
-    if ((double)B * (double)H > 2.0e9) return KDA_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, g, beta, S, o};
-    for (const void* p : ptrs)
-        if (!aligned16(p)) return KDA_ERR_MISALIGNED;
-    const size_t es = elem_size(dtype);
-    const size_t n = (size_t)B * H;
-    const Range rs = range_of(S, n * dk * dv * sizeof(float));
-    const Range ro = range_of(o, n * dv * es);
-    const Range ins[] = {range_of(q, n * dk * es), range_of(k, n * dk * es), range_of(v, n * dv * es),
-                         range_of(g, n * dk * es), range_of(beta, n * es)};
-    if (overlaps(rs, ro)) return KDA_ERR_INVALID_ARG;
-    for (const Range& r : ins)
-        if (overlaps(rs, r) || overlaps(ro, r)) return KDA_ERR_INVALID_ARG;
-    kda::DecodeArgs a{q, k, v, g, beta, S, o, B, H, dk, dv, dtype, status_word_for_current_device()};
-    if (!a.status) return KDA_ERR_CUDA;
-    return kda::launch_decode(a, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return decode_impl(q, k, v, g, beta, S, 0, nullptr, o, B, H, dk, dv, dtype, stream);
+}
+
+int kda_decode_step_paged(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                          float* S_pool, int n_slots, const int* slots, void* o, int B, int H, int dk,
+                          int dv, int dtype, struct CUstream_st* stream) {
+    if (!slots) return KDA_ERR_INVALID_ARG;
+    return decode_impl(q, k, v, g, beta, S_pool, n_slots, slots, o, B, H, dk, dv, dtype, stream);
 }
 
 int kda_state_compose(const float* M, const float* S_in, const float* N, float* S_out, int count, int dk,

@@ -24,7 +24,7 @@ template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kDecodeThreads)
 kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                   const Tin* __restrict__ g, const Tin* __restrict__ beta, float* __restrict__ S,
-                  Tin* __restrict__ o) {
+                  Tin* __restrict__ o, int H, const int* __restrict__ slots, int n_slots, int* status) {
     constexpr int LPR = DV / 4;                    // threads per state row (float4 each)
     constexpr int RPP = kDecodeThreads / LPR;      // rows covered per pass
     constexpr int RPT = DK / RPP;                  // rows per thread
@@ -40,7 +40,17 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
     const int lane = tid & 31, warp = tid >> 5;
     const int c4 = tid % LPR, rg = tid / LPR;
     const size_t bh = blockIdx.x;
-    float4* Sv = reinterpret_cast<float4*>(S + bh * DK * DV);
+    size_t sidx = bh;   // state of this (b, h): S[b, h], or S[slots[b], h] of a pool
+    if (slots) {
+        const int sl = slots[bh / H];
+        if (sl < 0) return;                        // inactive sequence: nothing is read or written
+        if (sl >= n_slots) {
+            if (tid == 0) report_status(status, KDA_ERR_INVALID_ARG);
+            return;
+        }
+        sidx = (size_t)sl * H + bh % H;
+    }
+    float4* Sv = reinterpret_cast<float4*>(S + sidx * DK * DV);
 
     // Issue the state loads first: 16 B per thread per row, all independent.
     float4 s[RPT];
@@ -120,7 +130,8 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t s) {
     const unsigned grid = (unsigned)((size_t)a.B * a.H);
     kda_decode_kernel<Tin, DK, DV><<<grid, kDecodeThreads, 0, s>>>(
         static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
-        static_cast<const Tin*>(a.g), static_cast<const Tin*>(a.beta), a.S, static_cast<Tin*>(a.o));
+        static_cast<const Tin*>(a.g), static_cast<const Tin*>(a.beta), a.S, static_cast<Tin*>(a.o), a.H, a.slots,
+        a.n_slots, a.status);
     return cudaGetLastError();
 }
 

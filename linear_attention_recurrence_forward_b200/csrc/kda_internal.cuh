@@ -27,6 +27,10 @@ struct PrefillArgs {
     float* S_mid;                   // states every `interval` tokens [B, H, n_mid, dk, dv], or null
     int interval;                   // multiple of 64 when S_mid is set
     int n_mid;                      // T / interval when S_mid is set, else 0
+    // Packed variable-length sequences: when set, q, k, g, v, o are [T, H, d] with T the total
+    // token count, B the number of sequences, and sequence b = tokens cu_seqlens[b] .. [b+1]-1
+    // (device array of B + 1 ints, checked by the kernels).
+    const int* cu_seqlens;
 };
 
 struct DecodeArgs {
@@ -40,6 +44,10 @@ struct DecodeArgs {
     int B, H, dk, dv;
     int dtype;
     int* status;
+    // Paged states: when set, sequence b's state is S[slots[b]] of a pool of n_slots states per
+    // head ([n_slots, H, dk, dv]); slots[b] < 0 skips the sequence.
+    const int* slots;
+    int n_slots;
 };
 
 // Launchers: return cudaSuccess or the launch error.  Defined in their kernel's .cu file.

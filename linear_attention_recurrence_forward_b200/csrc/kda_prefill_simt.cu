@@ -24,8 +24,8 @@ template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kSimtThreads)
 kda_prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                         const Tin* __restrict__ g, const Tin* __restrict__ beta,
-                        const float* S0, Tin* __restrict__ o, float* ST, int T, int H,
-                        float* S_mid, int interval, int n_mid) {
+                        const float* S0, Tin* __restrict__ o, float* ST, int T_all, int H,
+                        float* S_mid, int interval, int n_mid, const int* __restrict__ cu_seqlens, int* status) {
     constexpr int RPT = DK / kRpp;  // rows per thread (4 or 2)
     constexpr int NW = kSimtThreads / 32;
     constexpr int NSLICE = DV / kSlice;
@@ -40,6 +40,16 @@ kda_prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, co
     const size_t bh = blockIdx.x / NSLICE;
     const int b = (int)(bh / H), h = (int)(bh % H);
     const int col0 = slice * kSlice;
+    // tokens of this sequence: rows base .. base + T - 1 of the token axis
+    size_t base = (size_t)b * T_all;
+    int T = T_all;
+    if (cu_seqlens) {
+        const int s0 = cu_seqlens[b], s1 = cu_seqlens[b + 1];
+        const bool valid = 0 <= s0 && s0 <= s1 && s1 <= T_all;
+        if (!valid && threadIdx.x == 0) report_status(status, KDA_ERR_INVALID_ARG);
+        base = valid ? (size_t)s0 : 0;
+        T = valid ? s1 - s0 : 0;
+    }
 
     float4 s[RPT];
 #pragma unroll
@@ -50,7 +60,7 @@ kda_prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, co
     }
 
     auto stage = [&](int t, int buf) {
-        const size_t row = ((size_t)b * T + t) * H + h;
+        const size_t row = (base + t) * H + h;
         if (tid < DK) {
             qs[buf][tid] = load_elem(q, row * DK + tid);
             ks[buf][tid] = load_elem(k, row * DK + tid);
@@ -109,7 +119,7 @@ kda_prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, co
                 u.z = bt * (vs[buf][4 * lane + 2] - a.z);
                 u.w = bt * (vs[buf][4 * lane + 3] - a.w);
                 us[lane] = u;
-                const size_t oo = (((size_t)b * T + t) * H + h) * DV + col0 + 4 * lane;
+                const size_t oo = ((base + t) * H + h) * DV + col0 + 4 * lane;
                 store_elem(o, oo + 0, bb.x + kq * u.x);
                 store_elem(o, oo + 1, bb.y + kq * u.y);
                 store_elem(o, oo + 2, bb.z + kq * u.z);
@@ -148,7 +158,7 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s) {
     kda_prefill_simt_kernel<Tin, DK, DV><<<grid, kSimtThreads, 0, s>>>(
         static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
         static_cast<const Tin*>(a.g), static_cast<const Tin*>(a.beta), a.S0, static_cast<Tin*>(a.o),
-        a.ST, a.T, a.H, a.S_mid, a.interval, a.n_mid);
+        a.ST, a.T, a.H, a.S_mid, a.interval, a.n_mid, a.cu_seqlens, a.status);
     return cudaGetLastError();
 }
 

@@ -95,12 +95,14 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct TcParams {
     const __nv_bfloat16* beta;
     const float* S0;
+    __nv_bfloat16* o;               // for the per-row stores of a packed sequence's partial last chunk
     float* ST;
     int* status;
     unsigned long long timeout_ns;  // limit of every mbarrier wait
     int skip_handoff;               // test hook: never signal the first KQ hand-off
     float* S_mid;                   // state after every `interval` tokens, or null
     int interval, n_mid;
+    const int* cu_seqlens;          // packed sequences (B sequences over T tokens), or null
     int B, T, H;
 };
 
@@ -239,12 +241,27 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __shared__ __align__(16) float s_qsum[4][kD];      // g summed over each 16-token quarter
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    auto tid_is_zero = [&]() { return tid == 0; };
     const int quarter = warp & 3;              // TMEM lane quarter this warp may access
     const bool is_prep = warp < 8;
     const int colhalf = (warp >> 2) & 1;       // which 64 columns of a 128-wide result (per group)
     const int bh = blockIdx.x;
     const int b = bh / p.H, h = bh % p.H;
-    const int T = p.T;
+    // This CTA's tokens: rows tok0 .. tok0 + T - 1 of batch entry bmap of the tensor maps, i.e.
+    // [B, T, H, d] as laid out, or sequence b of packed sequences (maps with one batch entry of
+    // all tokens; offsets from cu_seqlens, checked here: an invalid range is reported and
+    // processed as empty)
+    const bool packed = p.cu_seqlens != nullptr;
+    int tok0 = 0, bmap = b, T = p.T;
+    if (packed) {
+        const int s0 = p.cu_seqlens[b], s1 = p.cu_seqlens[b + 1];
+        const bool valid = 0 <= s0 && s0 <= s1 && s1 <= p.T;
+        if (!valid && tid_is_zero()) report_status(p.status, KDA_ERR_INVALID_ARG);
+        tok0 = valid ? s0 : 0;
+        bmap = 0;
+        T = valid ? s1 - s0 : 0;
+    }
+    const size_t row0 = (size_t)bmap * p.T + tok0;   // token-axis row of this CTA's first token
     const int nchunks = (T + kC - 1) / kC;
 
     if (tid == 0) {
@@ -269,15 +286,15 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         mbar_arrive_expect_tx(&bar_qkg, 3u * 16384u);
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-            tma_load_4d(sm + OFF_RAW_Q + x * 8192, &tm_q, &bar_qkg, 64 * x, h, chunk * kC, b);
-            tma_load_4d(sm + OFF_RAW_K + x * 8192, &tm_k, &bar_qkg, 64 * x, h, chunk * kC, b);
-            tma_load_4d(sm + OFF_RAW_G + x * 8192, &tm_g, &bar_qkg, 64 * x, h, chunk * kC, b);
+            tma_load_4d(sm + OFF_RAW_Q + x * 8192, &tm_q, &bar_qkg, 64 * x, h, tok0 + chunk * kC, bmap);
+            tma_load_4d(sm + OFF_RAW_K + x * 8192, &tm_k, &bar_qkg, 64 * x, h, tok0 + chunk * kC, bmap);
+            tma_load_4d(sm + OFF_RAW_G + x * 8192, &tm_g, &bar_qkg, 64 * x, h, tok0 + chunk * kC, bmap);
         }
     };
     auto load_v = [&](int chunk) {
         mbar_arrive_expect_tx(&bar_v, 16384u);
 #pragma unroll
-        for (int x = 0; x < 2; ++x) tma_load_4d(sm + OFF_V + x * 8192, &tm_v, &bar_v, 64 * x, h, chunk * kC, b);
+        for (int x = 0; x < 2; ++x) tma_load_4d(sm + OFF_V + x * 8192, &tm_v, &bar_v, 64 * x, h, tok0 + chunk * kC, bmap);
     };
 
     bool ok = true;
@@ -303,7 +320,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const unsigned short* beta_bits = reinterpret_cast<const unsigned short*>(p.beta);
         auto fetch_beta = [&](int chunk) -> unsigned short {
             const int t = chunk * kC + ptid;
-            return (ptid < kC && t < T) ? beta_bits[((size_t)b * T + t) * p.H + h] : (unsigned short)0;
+            return (ptid < kC && t < T) ? beta_bits[(row0 + t) * p.H + h] : (unsigned short)0;
         };
         unsigned short beta_next = fetch_beta(0);
         for (int chunk = 0; chunk < nchunks; ++chunk) {
@@ -315,12 +332,14 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (ok && ptid == kIssuer) pending = -1;
             // ---- P2: Gam = in-chunk prefix sum of g in fp32: the running sum over this quarter,
             // then the totals of the quarters before it
+            const int nvalid = min(kC, T - chunk * kC);   // rows past it are padding: g = q = k = 0
             float gam[16][2];
             {
                 float a0 = 0.f, a1 = 0.f;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_G + sw128_offset(16 * tq + i, ch0, 8192));
+                    uint32_t w = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_G + sw128_offset(16 * tq + i, ch0, 8192));
+                    if (16 * tq + i >= nvalid) w = 0u;
                     a0 += __uint_as_float(w << 16);
                     a1 += __uint_as_float(w & 0xFFFF0000u);
                     gam[i][0] = a0;
@@ -384,8 +403,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int i = 0; i < 16; ++i) {
                     const int t = 16 * tq + i;
                     const int rq = 64 * hq + (t & 31), rk = rq + 32;   // MMA1 rows [Qt0;Kt0;Qt1;Kt1]
-                    const uint32_t qw = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_Q + sw128_offset(t, ch0, 8192));
-                    const uint32_t kw = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_K + sw128_offset(t, ch0, 8192));
+                    uint32_t qw = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_Q + sw128_offset(t, ch0, 8192));
+                    uint32_t kw = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_K + sw128_offset(t, ch0, 8192));
+                    if (t >= nvalid) qw = kw = 0u;
                     const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xFFFF0000u);
                     const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
                     const float x0 = fmaf(gam[i][0], kLog2e, -gmL[0]);
@@ -731,22 +751,35 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         __stcs(reinterpret_cast<float4*>(dst + j), make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]));
                 }
             }
+            // A packed sequence's partial last chunk is written row by row: the rows past its end
+            // belong to the next sequence, which a tile store would overwrite
+            const bool row_stores = packed && t0 + kC > T;
             if ((quarter & 1) == 0) {
                 const int r = 32 * (quarter >> 1) + lane;   // token row of the chunk
                 float ov[64];
                 tmem_ld64(tlane + TM_C + 64 * colhalf, ov);   // warp-collective
+                if (row_stores) {
+                    if (t0 + r < T) {
+                        uint4* orow = reinterpret_cast<uint4*>(p.o + ((row0 + t0 + r) * p.H + h) * kD + 64 * colhalf);
 #pragma unroll
-                for (int j = 0; j < 64; j += 8)
-                    *reinterpret_cast<uint4*>(sm + OFF_V + sw128_offset(r, 64 * colhalf + j, 8192)) = pack8(ov + j);
+                        for (int j = 0; j < 8; ++j) orow[j] = pack8(ov + 8 * j);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 64; j += 8)
+                        *reinterpret_cast<uint4*>(sm + OFF_V + sw128_offset(r, 64 * colhalf + j, 8192)) = pack8(ov + j);
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
             named_bar_sync(kBarSerial, kSerialThreads);
             if (stid == 0) {
-                // rows past T are clipped by the tensor map
-                tma_store_4d(&tm_o, sm + OFF_V, 0, h, t0, b);
-                tma_store_4d(&tm_o, sm + OFF_V + 8192, 64, h, t0, b);
-                bulk_commit_group();
+                // rows past the tensor's T are clipped by the tensor map
+                if (!row_stores) {
+                    tma_store_4d(&tm_o, sm + OFF_V, 0, h, tok0 + t0, bmap);
+                    tma_store_4d(&tm_o, sm + OFF_V + 8192, 64, h, tok0 + t0, bmap);
+                    bulk_commit_group();
+                }
                 if (chunk + 1 < nchunks) {
                     bulk_wait_read_all();   // the staged O is read: the next v may land on it
                     load_v(chunk + 1);
@@ -832,12 +865,15 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
         }
     }
     CUtensorMap mq, mk, mg, mv, mo;
-    if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
-        !make_map(&mg, a.g, a.B, a.T, a.H) || !make_map(&mv, a.v, a.B, a.T, a.H) ||
-        !make_map(&mo, a.o, a.B, a.T, a.H))
+    // packed sequences: one batch entry holding all T tokens
+    const int mb = a.cu_seqlens ? 1 : a.B;
+    if (!make_map(&mq, a.q, mb, a.T, a.H) || !make_map(&mk, a.k, mb, a.T, a.H) ||
+        !make_map(&mg, a.g, mb, a.T, a.H) || !make_map(&mv, a.v, mb, a.T, a.H) ||
+        !make_map(&mo, a.o, mb, a.T, a.H))
         return cudaErrorInvalidValue;
-    TcParams prm{static_cast<const __nv_bfloat16*>(a.beta), a.S0, a.ST,
-                 a.status, a.timeout_ns, a.skip_handoff, a.S_mid, a.interval, a.n_mid, a.B, a.T, a.H};
+    TcParams prm{static_cast<const __nv_bfloat16*>(a.beta), a.S0, static_cast<__nv_bfloat16*>(a.o), a.ST,
+                 a.status, a.timeout_ns, a.skip_handoff, a.S_mid, a.interval, a.n_mid, a.cu_seqlens,
+                 a.B, a.T, a.H};
     kda_prefill_tc_kernel<<<(unsigned)((size_t)a.B * a.H), kThreads, SMEM_DYN, s>>>(mq, mk, mg, mv, mo, prm);
     return cudaGetLastError();
 }
