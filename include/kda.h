@@ -145,6 +145,25 @@ KDA_API int kda_decode_step(const void* q, const void* k, const void* v, const v
                     int dtype, struct CUstream_st* stream);
 
 /*
+ * kda_forward_chunked_fused -- kda_forward_chunked with the gate and normalisation prologue fused
+ * into the kernels' load stage, so no separate elementwise pass over q, k, g and beta is needed:
+ *
+ *   g    = -5 * sigmoid(z_g)           per channel (the bounded scaled-sigmoid log-decay with
+ *                                      lower bound -5: Kimi K3 skill card (skillsmp.com), quick facts)
+ *   beta = sigmoid(z_beta)             per token and head
+ *   q, k = q_raw / |q_raw|, k_raw / |k_raw|   (L2 over the head dimension; a zero row stays zero)
+ *
+ * then exactly the recurrence of kda_forward_chunked.  Layouts, dtypes, sizes and rules as for
+ * kda_forward_chunked_impl with (q_raw, k_raw, v, z_g, z_beta) in the places of (q, k, v, g, beta).
+ * The tensor-core kernel forms sigmoid and the inverse norms with the hardware's approximate
+ * exponential, reciprocal and reciprocal square root (fp32, relative error ~1e-6); the fp32
+ * kernel with expf and rsqrtf.
+ */
+KDA_API int kda_forward_chunked_fused(const void* q_raw, const void* k_raw, const void* v, const void* z_g,
+                                      const void* z_beta, const float* S0, void* o, float* S_T, int B, int T,
+                                      int H, int dk, int dv, int dtype, int impl, struct CUstream_st* stream);
+
+/*
  * kda_forward_varlen -- prefill over packed sequences of different lengths (continuous batching).
  *
  * N sequences stored back to back along the token axis (the layout a paged serving engine

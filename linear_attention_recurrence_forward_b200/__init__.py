@@ -26,6 +26,7 @@ __all__ = [
     "kda_forward_chunked_states",
     "kda_decode_step",
     "kda_forward_varlen",
+    "kda_forward_chunked_fused",
     "kda_decode_step_paged",
     "kda_state_compose",
     "kda_get_device_status",
@@ -79,6 +80,8 @@ def lib() -> ctypes.CDLL:
         L.kda_forward_chunked_states.restype = I
         L.kda_state_compose.argtypes = [P, P, P, P, I, I, I, P]
         L.kda_state_compose.restype = I
+        L.kda_forward_chunked_fused.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P]
+        L.kda_forward_chunked_fused.restype = I
         L.kda_forward_varlen.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P]
         L.kda_forward_varlen.restype = I
         L.kda_decode_step_paged.argtypes = [P, P, P, P, P, P, I, P, P, I, I, I, I, I, P]
@@ -218,6 +221,37 @@ def kda_decode_step(q, k, v, g, beta, S, *, o=None, stream=None):
     if rc != 0:
         raise KdaError("kda_decode_step", rc)
     return o
+
+
+def kda_forward_chunked_fused(q_raw, k_raw, v, z_g, z_beta, S0=None, *, o=None, S_T=None,
+                              return_state: bool = True, impl: str = "auto", stream=None):
+    """Prefill with the prologue in the kernels: g = -5 sigmoid(z_g), beta = sigmoid(z_beta), q and k
+    L2-normalised over the head dimension.  Same layouts as kda_forward_chunked."""
+    B, T, H, dk = q_raw.shape
+    dv = v.shape[-1]
+    dev, dt = q_raw.device, q_raw.dtype
+    if dt not in DTYPE:
+        raise ValueError(f"unsupported dtype {dt}")
+    for name, t, shape in (("q_raw", q_raw, (B, T, H, dk)), ("k_raw", k_raw, (B, T, H, dk)),
+                           ("v", v, (B, T, H, dv)), ("z_g", z_g, (B, T, H, dk)), ("z_beta", z_beta, (B, T, H))):
+        _check(t, name, shape, dt, dev)
+    if S0 is not None:
+        _check(S0, "S0", (B, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    else:
+        _check(o, "o", (B, T, H, dv), dt, dev)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    elif S_T is not None:
+        _check(S_T, "S_T", (B, H, dk, dv), torch.float32, dev)
+    with torch.cuda.device(dev):
+        rc = lib().kda_forward_chunked_fused(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(z_g), _ptr(z_beta), _ptr(S0),
+                                             _ptr(o), _ptr(S_T), B, T, H, dk, dv, DTYPE[dt], IMPL[impl],
+                                             _stream_handle(stream))
+    if rc != 0:
+        raise KdaError("kda_forward_chunked_fused", rc)
+    return o, S_T
 
 
 def kda_forward_varlen(q, k, v, g, beta, cu_seqlens, S0=None, *, o=None, S_T=None, return_state: bool = True,

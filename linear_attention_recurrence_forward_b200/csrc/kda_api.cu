@@ -116,7 +116,7 @@ int validate_states(const void* q, const void* k, const void* v, const void* g, 
 int forward_impl(const void* q, const void* k, const void* v, const void* g, const void* beta,
                  const float* S0, void* o, float* ST, int B, int T, int H, int dk, int dv, int dtype,
                  int impl, cudaStream_t stream, float* S_mid = nullptr, int interval = 0,
-                 const int* cu_seqlens = nullptr) {
+                 const int* cu_seqlens = nullptr, int fused = 0) {
     if (impl != KDA_IMPL_AUTO && impl != KDA_IMPL_TCGEN05 && impl != KDA_IMPL_SIMT)
         return KDA_ERR_INVALID_ARG;
     // packed sequences: the activations are one batch entry of T tokens, the states B entries
@@ -137,7 +137,7 @@ int forward_impl(const void* q, const void* k, const void* v, const void* g, con
     }
     kda::PrefillArgs a{q, k, v, g, beta, S0, o, ST, B, T, H, dk, dv, dtype, nullptr,
                        g_timeout_ns.load(), g_skip_handoff.load(), n_mid > 0 ? S_mid : nullptr,
-                       interval, n_mid, cu_seqlens};
+                       interval, n_mid, cu_seqlens, fused};
     const bool tc_ok = kda::prefill_tc_supports(a);
     if (impl == KDA_IMPL_TCGEN05 && !tc_ok) return KDA_ERR_UNSUPPORTED;
     if (T == 0) {
@@ -212,6 +212,13 @@ int kda_forward_chunked_states(const void* q, const void* k, const void* v, cons
     if (interval <= 0) return KDA_ERR_INVALID_ARG;
     return forward_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, dtype, impl, stream, S_mid,
                         interval);
+}
+
+int kda_forward_chunked_fused(const void* q_raw, const void* k_raw, const void* v, const void* z_g,
+                              const void* z_beta, const float* S0, void* o, float* S_T, int B, int T, int H,
+                              int dk, int dv, int dtype, int impl, struct CUstream_st* stream) {
+    return forward_impl(q_raw, k_raw, v, z_g, z_beta, S0, o, S_T, B, T, H, dk, dv, dtype, impl, stream, nullptr,
+                        0, nullptr, 1);
 }
 
 int kda_forward_varlen(const void* q, const void* k, const void* v, const void* g, const void* beta,

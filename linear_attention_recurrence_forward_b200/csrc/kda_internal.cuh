@@ -31,6 +31,10 @@ struct PrefillArgs {
     // token count, B the number of sequences, and sequence b = tokens cu_seqlens[b] .. [b+1]-1
     // (device array of B + 1 ints, checked by the kernels).
     const int* cu_seqlens;
+    // Gate and normalisation prologue: q and k are raw (each kernel L2-normalises them over the
+    // head dimension), g holds the decay logit z (g = -5 sigmoid(z)) and beta the write logit
+    // (beta = sigmoid)
+    int fused;
 };
 
 struct DecodeArgs {

@@ -25,7 +25,8 @@ __global__ void __launch_bounds__(kSimtThreads)
 kda_prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                         const Tin* __restrict__ g, const Tin* __restrict__ beta,
                         const float* S0, Tin* __restrict__ o, float* ST, int T_all, int H,
-                        float* S_mid, int interval, int n_mid, const int* __restrict__ cu_seqlens, int* status) {
+                        float* S_mid, int interval, int n_mid, const int* __restrict__ cu_seqlens, int* status,
+                        int fused) {
     constexpr int RPT = DK / kRpp;  // rows per thread (4 or 2)
     constexpr int NW = kSimtThreads / 32;
     constexpr int NSLICE = DV / kSlice;
@@ -33,6 +34,8 @@ kda_prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, co
     __shared__ float qs[2][DK], ks[2][DK], es[2][DK], vs[2][kSlice], bs[2];
     __shared__ float4 red_a[NW][kLpr], red_b[NW][kLpr];
     __shared__ float4 us[kLpr];
+    __shared__ float qss[2][DK / 32], kss[2][DK / 32];   // prologue: per-warp sums of q^2, k^2
+    __shared__ float s_invk[2];                          // prologue: 1/|k| of the token
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int c4 = tid % kLpr, rg = tid / kLpr;
@@ -62,13 +65,27 @@ kda_prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, co
     auto stage = [&](int t, int buf) {
         const size_t row = (base + t) * H + h;
         if (tid < DK) {
-            qs[buf][tid] = load_elem(q, row * DK + tid);
-            ks[buf][tid] = load_elem(k, row * DK + tid);
-            es[buf][tid] = expf(load_elem(g, row * DK + tid));
+            const float qv = load_elem(q, row * DK + tid), kv = load_elem(k, row * DK + tid);
+            qs[buf][tid] = qv;
+            ks[buf][tid] = kv;
+            float gv = load_elem(g, row * DK + tid);
+            if (fused) {
+                // g = -5 sigmoid(z); the q and k norms as per-warp partial sums (full warps here)
+                gv = -5.f / (1.f + expf(-gv));
+                float sq = qv * qv, sk = kv * kv;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                    sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                }
+                if (lane == 0) { qss[buf][warp] = sq; kss[buf][warp] = sk; }
+            }
+            es[buf][tid] = expf(gv);
         } else if (tid < DK + kSlice) {
             vs[buf][tid - DK] = load_elem(v, row * DV + col0 + (tid - DK));
         } else if (tid == DK + kSlice) {
-            bs[buf] = load_elem(beta, row);
+            const float bz = load_elem(beta, row);
+            bs[buf] = fused ? 1.f / (1.f + expf(-bz)) : bz;
         }
     };
 
@@ -104,6 +121,17 @@ kda_prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, co
             for (int i = lane; i < DK; i += 32) kq += ks[buf][i] * qs[buf][i];
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+            // prologue: the sums above used the raw q and k; scale by 1/|q| and 1/|k|
+            float inv_q = 1.f, inv_k = 1.f;
+            if (fused) {
+                float sq = 0.f, sk = 0.f;
+#pragma unroll
+                for (int w = 0; w < DK / 32; ++w) { sq += qss[buf][w]; sk += kss[buf][w]; }
+                inv_q = sq > 0.f ? rsqrtf(sq) : 0.f;
+                inv_k = sk > 0.f ? rsqrtf(sk) : 0.f;
+                kq *= inv_q * inv_k;
+                if (lane == 0) s_invk[buf] = inv_k;
+            }
             if (lane < kLpr) {
                 float4 a = red_a[0][lane], bb = red_b[0][lane];
 #pragma unroll
@@ -112,6 +140,8 @@ kda_prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, co
                     a.x += ta.x; a.y += ta.y; a.z += ta.z; a.w += ta.w;
                     bb.x += tb.x; bb.y += tb.y; bb.z += tb.z; bb.w += tb.w;
                 }
+                a.x *= inv_k; a.y *= inv_k; a.z *= inv_k; a.w *= inv_k;
+                bb.x *= inv_q; bb.y *= inv_q; bb.z *= inv_q; bb.w *= inv_q;
                 const float bt = bs[buf];
                 float4 u;
                 u.x = bt * (vs[buf][4 * lane + 0] - a.x);
@@ -128,9 +158,10 @@ kda_prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, co
         }
         __syncthreads();
         const float4 u = us[c4];
+        const float kscale = fused ? s_invk[buf] : 1.f;
 #pragma unroll
         for (int j = 0; j < RPT; ++j) {
-            const float kr = ks[buf][rg + j * kRpp];
+            const float kr = ks[buf][rg + j * kRpp] * kscale;
             s[j].x += kr * u.x; s[j].y += kr * u.y; s[j].z += kr * u.z; s[j].w += kr * u.w;
         }
         // the state after a multiple of the interval
@@ -158,7 +189,7 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s) {
     kda_prefill_simt_kernel<Tin, DK, DV><<<grid, kSimtThreads, 0, s>>>(
         static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
         static_cast<const Tin*>(a.g), static_cast<const Tin*>(a.beta), a.S0, static_cast<Tin*>(a.o),
-        a.ST, a.T, a.H, a.S_mid, a.interval, a.n_mid, a.cu_seqlens, a.status);
+        a.ST, a.T, a.H, a.S_mid, a.interval, a.n_mid, a.cu_seqlens, a.status, a.fused);
     return cudaGetLastError();
 }
 

@@ -103,6 +103,7 @@ struct TcParams {
     float* S_mid;                   // state after every `interval` tokens, or null
     int interval, n_mid;
     const int* cu_seqlens;          // packed sequences (B sequences over T tokens), or null
+    int fused;                      // 1: q, k raw (L2-normalised here), g and beta given as logits
     int B, T, H;
 };
 
@@ -192,6 +193,15 @@ __device__ __forceinline__ void mm16_acc(float out[2][4], const uint32_t ax[4], 
     }
 }
 
+__device__ __forceinline__ float ex2_approx(float x);
+// The gate prologue: beta = sigmoid(z) and the bounded log-decay g = -5 sigmoid(z) (the scaled
+// sigmoid with lower bound -5 of the skill card's quick facts).  1 + e^{-z} overflows to inf for
+// z << 0, which gives 0 (no decay / no write), the limit.
+__device__ __forceinline__ float sigmoid_fast(float z) { return __fdividef(1.f, 1.f + ex2_approx(-z * 1.4426950408889634f)); }
+__device__ __forceinline__ float log_decay_from_logit(float z) {
+    return __fdividef(-5.f, 1.f + ex2_approx(-z * 1.4426950408889634f));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -239,6 +249,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __shared__ __align__(16) float s_gamma[2][kD];     // e^{Gam_63} per channel, by chunk parity (float2 stores)
     __shared__ __align__(16) float s_refs[4][kD];      // Gam rows 16, 31, 48, 63
     __shared__ __align__(16) float s_qsum[4][kD];      // g summed over each 16-token quarter
+    __shared__ float s_norm[2 * kC];                   // with the prologue: 1/|q_t|, then 1/|k_t|
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     auto tid_is_zero = [&]() { return tid == 0; };
@@ -326,7 +337,11 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         for (int chunk = 0; chunk < nchunks; ++chunk) {
             const uint32_t par = chunk & 1, ppar = par ^ 1u;
             // ---- P1: beta; this chunk's q, k, g
-            if (ptid < kC) s_beta[ptid] = __uint_as_float((uint32_t)beta_next << 16);
+            if (ptid < kC) {
+                const float bz = __uint_as_float((uint32_t)beta_next << 16);
+                // with the prologue beta is a logit; a padding token keeps beta = 0
+                s_beta[ptid] = p.fused ? (chunk * kC + ptid < T ? sigmoid_fast(bz) : 0.f) : bz;
+            }
             if (chunk + 1 < nchunks) beta_next = fetch_beta(chunk + 1);
             ok = mbar_wait(&bar_qkg, par, p.timeout_ns);   // every thread: its own view of the TMA data
             if (ok && ptid == kIssuer) pending = -1;
@@ -338,10 +353,12 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 float a0 = 0.f, a1 = 0.f;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    uint32_t w = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_G + sw128_offset(16 * tq + i, ch0, 8192));
-                    if (16 * tq + i >= nvalid) w = 0u;
-                    a0 += __uint_as_float(w << 16);
-                    a1 += __uint_as_float(w & 0xFFFF0000u);
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_G + sw128_offset(16 * tq + i, ch0, 8192));
+                    float g0 = __uint_as_float(w << 16), g1 = __uint_as_float(w & 0xFFFF0000u);
+                    if (p.fused) { g0 = log_decay_from_logit(g0); g1 = log_decay_from_logit(g1); }
+                    if (16 * tq + i >= nvalid) g0 = g1 = 0.f;
+                    a0 += g0;
+                    a1 += g1;
                     gam[i][0] = a0;
                     gam[i][1] = a1;
                 }
@@ -349,6 +366,25 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             ok = named_bar_and(kBarPrep, kPrepThreads, ok);
             if (!ok) break;
+            if (p.fused) {
+                // 1/|x| of every q and k row of the chunk (row = thread/2, 64 channels per thread)
+                const int row = ptid >> 1, half = ptid & 1, t = row & (kC - 1);
+                const uint8_t* tile = sm + (row < kC ? OFF_RAW_Q : OFF_RAW_K) + half * 8192 + t * 128;
+                float ss = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint4 w4 = *reinterpret_cast<const uint4*>(tile + ((j ^ (t & 7)) << 4));
+                    const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float lo = __uint_as_float(wv[e] << 16), hi = __uint_as_float(wv[e] & 0xFFFF0000u);
+                        ss = fmaf(lo, lo, ss);
+                        ss = fmaf(hi, hi, ss);
+                    }
+                }
+                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                if (half == 0) s_norm[row] = ss > 0.f ? rsqrtf(ss) : 0.f;
+            }
             {
                 float c0s = 0.f, c1s = 0.f;
 #pragma unroll 1
@@ -406,8 +442,12 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     uint32_t qw = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_Q + sw128_offset(t, ch0, 8192));
                     uint32_t kw = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_K + sw128_offset(t, ch0, 8192));
                     if (t >= nvalid) qw = kw = 0u;
-                    const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xFFFF0000u);
-                    const float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
+                    float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xFFFF0000u);
+                    float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
+                    if (p.fused) {
+                        const float qn = s_norm[t], kn = s_norm[kC + t];
+                        q0 *= qn; q1 *= qn; k0 *= kn; k1 *= kn;
+                    }
                     const float x0 = fmaf(gam[i][0], kLog2e, -gmL[0]);
                     const float x1 = fmaf(gam[i][1], kLog2e, -gmL[1]);
                     const float E0 = ex2_approx(x0), E1 = ex2_approx(x1);
@@ -873,7 +913,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
         return cudaErrorInvalidValue;
     TcParams prm{static_cast<const __nv_bfloat16*>(a.beta), a.S0, static_cast<__nv_bfloat16*>(a.o), a.ST,
                  a.status, a.timeout_ns, a.skip_handoff, a.S_mid, a.interval, a.n_mid, a.cu_seqlens,
-                 a.B, a.T, a.H};
+                 a.fused, a.B, a.T, a.H};
     kda_prefill_tc_kernel<<<(unsigned)((size_t)a.B * a.H), kThreads, SMEM_DYN, s>>>(mq, mk, mg, mv, mo, prm);
     return cudaGetLastError();
 }

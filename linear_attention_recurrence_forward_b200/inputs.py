@@ -36,6 +36,7 @@ __all__ = [
     "DECODE_CONFIG",
     "make_prefill_inputs",
     "make_decode_inputs",
+    "make_prefill_raw_inputs",
     "torch_dtype",
 ]
 
@@ -132,6 +133,27 @@ def make_prefill_inputs(B: int, T: int, H: int, dk: int, dv: int, dtype: str = "
     if s0_std > 0.0:
         S0 = _normal((B, H, dk, dv), gen, device).mul_(s0_std)
     return q, k, v, g, beta, S0
+
+
+def make_prefill_raw_inputs(B: int, T: int, H: int, dk: int, dv: int, dtype: str = "bf16",
+                            seed: int = 0, s0_std: float = 0.0, zg_mean: float = 0.0,
+                            device: str = "cpu", gen: Optional[torch.Generator] = None):
+    """The same draws as make_prefill_inputs before any transformation: (q_raw, k_raw, v, z_g,
+    z_beta, S0) with q_raw, k_raw ~ N(0, 1) (not normalised), z_g ~ N(zg_mean, 1), z_beta ~ N(0, 1),
+    all rounded to the dtype; for the prologue-fused prefill."""
+    if gen is None:
+        gen = torch.Generator(device=device)
+        gen.manual_seed(seed)
+    dt = torch_dtype(dtype)
+    q = _normal((B, T, H, dk), gen, device).to(dt)
+    k = _normal((B, T, H, dk), gen, device).to(dt)
+    v = _normal((B, T, H, dv), gen, device).to(dt)
+    z_g = _normal((B, T, H, dk), gen, device, mean=zg_mean).to(dt)
+    z_beta = _normal((B, T, H), gen, device).to(dt)
+    S0 = None
+    if s0_std > 0.0:
+        S0 = _normal((B, H, dk, dv), gen, device).mul_(s0_std)
+    return q, k, v, z_g, z_beta, S0
 
 
 def make_config_inputs(cfg: KdaConfig, device: str = "cpu"):

@@ -115,6 +115,31 @@ def forward(q, k, v, g, beta, S0=None, nthreads: int = 0, lib: ctypes.CDLL = Non
     return o, ST
 
 
+def prologue(q_raw, k_raw, z_g, z_beta):
+    """The gate and normalisation prologue in fp64: (q, k, g, beta).
+
+    g = -5 * sigmoid(z_g): the bounded scaled-sigmoid log-decay with lower bound -5 (skill card
+    (skillsmp.com), quick facts); beta = sigmoid(z_beta) (reading: one logit per token and head);
+    q, k divided by their L2 norm over the head dimension (the input recipe of the workloads; a
+    zero row stays zero).
+    """
+    q_raw, k_raw, z_g, z_beta = (to_f64(x) for x in (q_raw, k_raw, z_g, z_beta))
+
+    def unit(x):
+        n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+        return np.divide(x, n, out=np.zeros_like(x), where=n > 0)
+
+    g = -5.0 / (1.0 + np.exp(-z_g))
+    beta = 1.0 / (1.0 + np.exp(-z_beta))
+    return unit(q_raw), unit(k_raw), g, beta
+
+
+def forward_fused(q_raw, k_raw, v, z_g, z_beta, S0=None, nthreads: int = 0, lib: ctypes.CDLL = None):
+    """The prologue, then forward(): what the prologue-fused prefill computes."""
+    q, k, g, beta = prologue(q_raw, k_raw, z_g, z_beta)
+    return forward(q, k, v, g, beta, S0, nthreads=nthreads, lib=lib)
+
+
 def forward_states(q, k, v, g, beta, S0=None, interval: int = 512, nthreads: int = 0,
                    lib: ctypes.CDLL = None):
     """forward() that also returns the state after every `interval` tokens.
