@@ -340,6 +340,32 @@ def run_ours(args):
                        "timed": "separately, after the headline region (rank 0's own device)"}
         del S_mid
 
+    # ---- the same prefill with the gate / normalisation prologue in the kernel, on raw inputs
+    fused_line = None
+    if not args.no_states:
+        from linear_attention_recurrence_forward_b200.inputs import make_prefill_raw_inputs
+        raw = make_prefill_raw_inputs(P["B"], P["T"], P["H"], P["dk"], P["dv"], P["dtype"], seed=3000 + rank,
+                                      s0_std=P["s0_std"], zg_mean=P["zg_mean"], device=str(dev))
+        for _ in range(2):
+            kda.kda_forward_chunked_fused(*raw[:5], raw[5], o=o, S_T=ST, stream=stream)
+        reps = max(3, min(args.steps, 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            kda.kda_forward_chunked_fused(*raw[:5], raw[5], o=o, S_T=ST, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if kda.kda_get_device_status() != 0:
+            raise RuntimeError("device status after the prologue-fused run")
+        f_ms = e0.elapsed_time(e1) / reps
+        fb = prefill_alg_bytes(P["B"], P["T"], P["H"], P["dk"], P["dv"])
+        fused_line = {"launch_ms": f_ms, "tokens_per_s": P["B"] * P["T"] / (f_ms / 1e3),
+                      "achieved_gbs": fb / (f_ms / 1e3) / 1e9, "launches": reps,
+                      "note": "raw q, k and gate logits in; g, beta and the q/k norms formed in the kernel "
+                              "(an unfused pipeline also reads and writes them once more in a separate pass)"}
+        del raw
+
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
     if args.no_e2e:
         e2e = None
@@ -386,6 +412,7 @@ def run_ours(args):
                                 "frac": dec_achieved / peak, "alg_bytes_per_launch": db_,
                                 "traffic": recorded_traffic("decode")}},
         "state_emission": states_line,
+        "fused_prologue": fused_line,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": 2 * args.steps,
