@@ -103,7 +103,6 @@ struct TcParams {
     float* S_mid;                   // state after every `interval` tokens, or null
     int interval, n_mid;
     const int* cu_seqlens;          // packed sequences (B sequences over T tokens), or null
-    int fused;                      // 1: q, k raw (L2-normalised here), g and beta given as logits
     int B, T, H;
 };
 
@@ -230,6 +229,9 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
 // 64-95, so that the products land in the TMEM lanes of the Qt rows.
 __device__ __forceinline__ int tp_row(int r) { return r < 32 ? r : r + 32; }
 
+// kFused: the gate and normalisation prologue (q, k raw; g, beta as logits).  kPacked: packed
+// variable-length sequences.  Compiled separately so that the plain path carries neither.
+template <bool kFused, bool kPacked>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_v,
@@ -262,9 +264,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // [B, T, H, d] as laid out, or sequence b of packed sequences (maps with one batch entry of
     // all tokens; offsets from cu_seqlens, checked here: an invalid range is reported and
     // processed as empty)
-    const bool packed = p.cu_seqlens != nullptr;
     int tok0 = 0, bmap = b, T = p.T;
-    if (packed) {
+    if (kPacked) {
         const int s0 = p.cu_seqlens[b], s1 = p.cu_seqlens[b + 1];
         const bool valid = 0 <= s0 && s0 <= s1 && s1 <= p.T;
         if (!valid && tid_is_zero()) report_status(p.status, KDA_ERR_INVALID_ARG);
@@ -340,14 +341,16 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (ptid < kC) {
                 const float bz = __uint_as_float((uint32_t)beta_next << 16);
                 // with the prologue beta is a logit; a padding token keeps beta = 0
-                s_beta[ptid] = p.fused ? (chunk * kC + ptid < T ? sigmoid_fast(bz) : 0.f) : bz;
+                s_beta[ptid] = kFused ? (chunk * kC + ptid < T ? sigmoid_fast(bz) : 0.f) : bz;
             }
             if (chunk + 1 < nchunks) beta_next = fetch_beta(chunk + 1);
             ok = mbar_wait(&bar_qkg, par, p.timeout_ns);   // every thread: its own view of the TMA data
             if (ok && ptid == kIssuer) pending = -1;
             // ---- P2: Gam = in-chunk prefix sum of g in fp32: the running sum over this quarter,
             // then the totals of the quarters before it
-            const int nvalid = min(kC, T - chunk * kC);   // rows past it are padding: g = q = k = 0
+            // rows past nvalid are padding: the tensor map reads zeros there for the [B, T, H, d] layout,
+            // but the next sequence's rows for packed sequences, and a zero logit is no zero gate
+            const int nvalid = min(kC, T - chunk * kC);
             float gam[16][2];
             {
                 float a0 = 0.f, a1 = 0.f;
@@ -355,8 +358,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int i = 0; i < 16; ++i) {
                     const uint32_t w = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_G + sw128_offset(16 * tq + i, ch0, 8192));
                     float g0 = __uint_as_float(w << 16), g1 = __uint_as_float(w & 0xFFFF0000u);
-                    if (p.fused) { g0 = log_decay_from_logit(g0); g1 = log_decay_from_logit(g1); }
-                    if (16 * tq + i >= nvalid) g0 = g1 = 0.f;
+                    if (kFused) { g0 = log_decay_from_logit(g0); g1 = log_decay_from_logit(g1); }
+                    if ((kFused || kPacked) && 16 * tq + i >= nvalid) g0 = g1 = 0.f;
                     a0 += g0;
                     a1 += g1;
                     gam[i][0] = a0;
@@ -366,7 +369,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             ok = named_bar_and(kBarPrep, kPrepThreads, ok);
             if (!ok) break;
-            if (p.fused) {
+            if (kFused) {
                 // 1/|x| of every q and k row of the chunk (row = thread/2, 64 channels per thread)
                 const int row = ptid >> 1, half = ptid & 1, t = row & (kC - 1);
                 const uint8_t* tile = sm + (row < kC ? OFF_RAW_Q : OFF_RAW_K) + half * 8192 + t * 128;
@@ -441,10 +444,10 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     const int rq = 64 * hq + (t & 31), rk = rq + 32;   // MMA1 rows [Qt0;Kt0;Qt1;Kt1]
                     uint32_t qw = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_Q + sw128_offset(t, ch0, 8192));
                     uint32_t kw = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_K + sw128_offset(t, ch0, 8192));
-                    if (t >= nvalid) qw = kw = 0u;
+                    if (kPacked && t >= nvalid) qw = kw = 0u;
                     float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xFFFF0000u);
                     float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
-                    if (p.fused) {
+                    if (kFused) {
                         const float qn = s_norm[t], kn = s_norm[kC + t];
                         q0 *= qn; q1 *= qn; k0 *= kn; k1 *= kn;
                     }
@@ -793,7 +796,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             // A packed sequence's partial last chunk is written row by row: the rows past its end
             // belong to the next sequence, which a tile store would overwrite
-            const bool row_stores = packed && t0 + kC > T;
+            const bool row_stores = kPacked && t0 + kC > T;
             if ((quarter & 1) == 0) {
                 const int r = 32 * (quarter >> 1) + lane;   // token row of the chunk
                 float ov[64];
@@ -899,8 +902,11 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     {
         std::lock_guard<std::mutex> lock(mu);
         if (dev < 64 && !attr_set[dev]) {
-            e = cudaFuncSetAttribute(kda_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
-            if (e != cudaSuccess) return e;
+            for (const void* fn : {(const void*)kda_prefill_tc_kernel<false, false>, (const void*)kda_prefill_tc_kernel<true, false>,
+                                   (const void*)kda_prefill_tc_kernel<false, true>, (const void*)kda_prefill_tc_kernel<true, true>}) {
+                e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
+                if (e != cudaSuccess) return e;
+            }
             attr_set[dev] = true;
         }
     }
@@ -913,8 +919,15 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
         return cudaErrorInvalidValue;
     TcParams prm{static_cast<const __nv_bfloat16*>(a.beta), a.S0, static_cast<__nv_bfloat16*>(a.o), a.ST,
                  a.status, a.timeout_ns, a.skip_handoff, a.S_mid, a.interval, a.n_mid, a.cu_seqlens,
-                 a.fused, a.B, a.T, a.H};
-    kda_prefill_tc_kernel<<<(unsigned)((size_t)a.B * a.H), kThreads, SMEM_DYN, s>>>(mq, mk, mg, mv, mo, prm);
+                 a.B, a.T, a.H};
+    const unsigned grid = (unsigned)((size_t)a.B * a.H);
+    if (a.cu_seqlens) {
+        if (a.fused) kda_prefill_tc_kernel<true, true><<<grid, kThreads, SMEM_DYN, s>>>(mq, mk, mg, mv, mo, prm);
+        else kda_prefill_tc_kernel<false, true><<<grid, kThreads, SMEM_DYN, s>>>(mq, mk, mg, mv, mo, prm);
+    } else {
+        if (a.fused) kda_prefill_tc_kernel<true, false><<<grid, kThreads, SMEM_DYN, s>>>(mq, mk, mg, mv, mo, prm);
+        else kda_prefill_tc_kernel<false, false><<<grid, kThreads, SMEM_DYN, s>>>(mq, mk, mg, mv, mo, prm);
+    }
     return cudaGetLastError();
 }
 
