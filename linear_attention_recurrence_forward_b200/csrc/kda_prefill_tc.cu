@@ -229,6 +229,45 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
 // 64-95, so that the products land in the TMEM lanes of the Qt rows.
 __device__ __forceinline__ int tp_row(int r) { return r < 32 ? r : r + 32; }
 
+// One warp's walk down block column J of X = (I + A)^-1 (its 8 output columns nt): for R = J+1 .. 3,
+// X_RJ = -X_RR (sum_{L=J}^{R-1} A_RL X_LJ) on warp-level bf16 tensor-core tiles with fp32 sums (bf16
+// operands here leave the output error unchanged in the chunk model).  Each X_LJ it needs is the
+// diagonal block (level 0's transposed copy) or one it has just formed, kept as a B fragment in
+// registers, so no other warp is waited for; T = X Diag(beta) entries are written as they are formed.
+template <int J>
+__device__ __forceinline__ void offdiag_column(const float* AF, const float* XF, const float* XT,
+                                               const float* beta, uint8_t* sm, int nt, int lane) {
+    const int g4 = lane >> 2, t4 = lane & 3;
+    uint32_t xb[3 - J][2];   // B fragments of X_LJ, L = J .. 2
+    load_b_frag(XT + (16 * J + 8 * nt) * kLd + 16 * J, kLd, g4, t4, xb[0]);
+    const int col = 16 * J + 8 * nt + 2 * t4;
+    const float b0 = beta[col], b1 = beta[col + 1];
+#pragma unroll
+    for (int R = J + 1; R < 4; ++R) {
+        float w[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int L = J; L < R; ++L) {
+            uint32_t af[4];
+            load_a_frag(AF + (16 * R) * kLd + 16 * L, kLd, g4, t4, af);
+            mma_16816(w, af, xb[L - J]);
+        }
+        // W as the B operand (its 16 rows are K) of X_RR W
+        const uint32_t wb[2] = {movmatrix_trans(pack_bf16x2(w[0], w[1])), movmatrix_trans(pack_bf16x2(w[2], w[3]))};
+        uint32_t ar[4];
+        load_a_frag(XF + (16 * R) * kLd + 16 * R, kLd, g4, t4, ar);
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_16816(x, ar, wb);
+        *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(16 * R + g4), col, 8192)) =
+            pack_bf16x2(-x[0] * b0, -x[1] * b1);
+        *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(16 * R + g4 + 8), col, 8192)) =
+            pack_bf16x2(-x[2] * b0, -x[3] * b1);
+        if (R < 3) {
+            xb[R - J][0] = movmatrix_trans(pack_bf16x2(-x[0], -x[1]));
+            xb[R - J][1] = movmatrix_trans(pack_bf16x2(-x[2], -x[3]));
+        }
+    }
+}
+
 // kFused: the gate and normalisation prologue (q, k raw; g, beta as logits).  kPacked: packed
 // variable-length sequences.  Compiled separately so that the plain path carries neither.
 template <bool kFused, bool kPacked>
@@ -587,54 +626,12 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
             }
             named_bar_sync(kBarPrep, kPrepThreads);
-            // X_RJ = -X_RR sum_{L=J}^{R-1} A_RL X_LJ by block distance d = R - J on warp-level bf16
-            // tensor-core tiles, fp32 accumulation (bf16 operands here leave the output error
-            // unchanged in the chunk model).  Warp 2*qb + nt: 8 output columns nt of block qb.
-            {
-                const int g4 = lane >> 2, t4 = lane & 3;
-                float* WS = reinterpret_cast<float*>(sm + OFF_WS) + warp * 8 * kLdS;
-#pragma unroll
-                for (int d = 1; d < 4; ++d) {
-                    if (warp < 2 * (4 - d)) {
-                        const int qb = warp >> 1, nt = warp & 1;
-                        const int R = qb + d, J = qb;
-                        float w[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                        for (int Lb = 0; Lb < 3; ++Lb) {
-                            if (Lb < d) {
-                                const int L = J + Lb;
-                                uint32_t af[4], bf[2];
-                                load_a_frag(AF + (16 * R) * kLd + 16 * L, kLd, g4, t4, af);
-                                load_b_frag(XT + (16 * J + 8 * nt) * kLd + 16 * L, kLd, g4, t4, bf);
-                                mma_16816(w, af, bf);
-                            }
-                        }
-                        WS[(2 * t4) * kLdS + g4] = w[0];
-                        WS[(2 * t4 + 1) * kLdS + g4] = w[1];
-                        WS[(2 * t4) * kLdS + g4 + 8] = w[2];
-                        WS[(2 * t4 + 1) * kLdS + g4 + 8] = w[3];
-                        __syncwarp();
-                        uint32_t af[4], bf[2];
-                        load_a_frag(XF + (16 * R) * kLd + 16 * R, kLd, g4, t4, af);
-                        load_b_frag(WS, kLdS, g4, t4, bf);
-                        float x[4] = {0.f, 0.f, 0.f, 0.f};
-                        mma_16816(x, af, bf);
-                        const int col = 16 * J + 8 * nt + 2 * t4;
-                        *reinterpret_cast<float2*>(XF + (16 * R + g4) * kLd + col) = make_float2(-x[0], -x[1]);
-                        *reinterpret_cast<float2*>(XF + (16 * R + g4 + 8) * kLd + col) = make_float2(-x[2], -x[3]);
-                        XT[col * kLd + 16 * R + g4] = -x[0];
-                        XT[(col + 1) * kLd + 16 * R + g4] = -x[1];
-                        XT[col * kLd + 16 * R + g4 + 8] = -x[2];
-                        XT[(col + 1) * kLd + 16 * R + g4 + 8] = -x[3];
-                        // T = X Diag(beta) for these entries
-                        const float b0 = s_beta[col], b1 = s_beta[col + 1];
-                        *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(16 * R + g4), col, 8192)) =
-                            pack_bf16x2(-x[0] * b0, -x[1] * b1);
-                        *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(16 * R + g4 + 8), col, 8192)) =
-                            pack_bf16x2(-x[2] * b0, -x[3] * b1);
-                    }
-                    named_bar_sync(kBarPrep, kPrepThreads);
-                }
+            // off-diagonal blocks, one block column per warp pair (8 output columns per warp)
+            if (warp < 6) {
+                const int nt = warp & 1;
+                if (warp < 2) offdiag_column<0>(AF, XF, XT, s_beta, sm, nt, lane);
+                else if (warp < 4) offdiag_column<1>(AF, XF, XT, s_beta, sm, nt, lane);
+                else offdiag_column<2>(AF, XF, XT, s_beta, sm, nt, lane);
             }
             fence_proxy_async_smem();
             named_bar_sync(kBarPrep, kPrepThreads);
