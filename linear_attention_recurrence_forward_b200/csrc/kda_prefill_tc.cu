@@ -53,7 +53,8 @@ constexpr int kThreads = 512;   // 16 warps
 constexpr int kPrepThreads = 256;
 constexpr int kSerialThreads = 256;
 constexpr uint32_t kBarPrep = 1, kBarSerial = 2;   // named hardware barriers
-constexpr int kIssuer = 0;                         // prep thread that issues its TMA loads and MMAs
+constexpr int kIssuer = 0;                         // prep thread that issues the first TMA load and signals
+constexpr int kMma1Issuer = 224;                   // prep thread that issues MMA1 (warp 7: lightest in the solve)
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
 constexpr uint32_t OFF_RAW_Q = 0;           // TMA destination, bf16 [64 tok][128], 2 boxes of 8 KB
@@ -284,7 +285,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
     // TMA / MMA completion barriers (one phase per chunk) and prep -> serial hand-offs.
     __shared__ uint64_t bar_qkg, bar_v, bar_ap, bar_c, bar_u, bar_os, bar_kq, bar_tpk;
-    __shared__ uint64_t bar_drain_p, bar_drain_s;
+    __shared__ uint64_t bar_drain_p, bar_drain_s, bar_drain_g;
     __shared__ uint32_t tmem_base_s;
     __shared__ __align__(16) float s_beta[kC];
     __shared__ __align__(16) float s_gamma[2][kD];     // e^{Gam_63} per channel, by chunk parity (float2 stores)
@@ -318,7 +319,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (tid == 0) {
         mbar_init(&bar_qkg, 1); mbar_init(&bar_v, 1); mbar_init(&bar_ap, 1);
         mbar_init(&bar_c, 1); mbar_init(&bar_u, 1); mbar_init(&bar_os, 1); mbar_init(&bar_kq, 1);
-        mbar_init(&bar_tpk, 1); mbar_init(&bar_drain_p, 1); mbar_init(&bar_drain_s, 1);
+        mbar_init(&bar_tpk, 1); mbar_init(&bar_drain_p, 1); mbar_init(&bar_drain_s, 1); mbar_init(&bar_drain_g, 1);
         fence_mbar_init();
         prefetch_tensormap(&tm_q); prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_g); prefetch_tensormap(&tm_v); prefetch_tensormap(&tm_o);
@@ -516,8 +517,14 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             fence_proxy_async_smem();
             tc_fence_before_sync();
             named_bar_sync(kBarPrep, kPrepThreads);
-            // A1, BB and KQ of this chunk are ready and its raw q, k, g consumed: the recurrence group's
-            // leader issues MMA1, MMA3 and the next chunk's loads
+            // KQ of this chunk is ready and its raw q, k, g consumed: the recurrence group's leader
+            // issues MMA3 and the next chunk's loads
+            // MMA1 (A and P of the chunk) straight from this group: it is on this group's path
+            if (ptid == kMma1Issuer) {
+                tc_fence_after_sync();
+                issue_mma<8, false, 16384, false, 12288>(tbase + TM_P, sb + OFF_A1, sb + OFF_BB, ID_MMA1, false);
+                mma_commit(&bar_ap);
+            }
             if (ptid == kIssuer && !(p.skip_handoff && chunk == 0)) mbar_arrive(&bar_kq);
             // ---- P4: Kb tile, P and A from TMEM, triangular solve, T tile
             if (chunk > 0) ok = mbar_wait(&bar_os, ppar, p.timeout_ns);  // T, P, Kb released
@@ -639,6 +646,10 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         if (!ok && ptid == 0) report_status(p.status, KDA_ERR_TIMEOUT);
         // drain: no MMA or TMA issued by this group may still be in flight
+        if (ptid == kMma1Issuer) {
+            mma_commit(&bar_drain_g);
+            if (!mbar_wait(&bar_drain_g, 0, p.timeout_ns)) report_status(p.status, KDA_ERR_TIMEOUT);
+        }
         if (ptid == kIssuer) {
             mma_commit(&bar_drain_p);
             if (!mbar_wait(&bar_drain_p, 0, p.timeout_ns)) report_status(p.status, KDA_ERR_TIMEOUT);
@@ -649,13 +660,10 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int stid = tid - kPrepThreads;                // 0..255
         int pending = -1;                                   // chunk whose v load is in flight
         int pending_qkg = -1;                               // last chunk whose q,k,g loads this leader issued
-        // Once the prep group has published chunk c's operand tiles (bar_kq): MMA1 (its A and P
-        // products, on the prep group's path, so first), MMA3 = [Qt0;Kt0;Qt1;Kt1] S, and the raw
-        // q, k, g of chunk c+1 into the buffers the prep group has finished reading.
+        // Once the prep group has published chunk c's operand tiles (bar_kq): MMA3 = [Qt0;Kt0;Qt1;Kt1] S
+        // and the raw q, k, g of chunk c+1 into the buffers the prep group has finished reading.
         auto issue_for_chunk = [&](int c) {
             tc_fence_after_sync();
-            issue_mma<8, false, 16384, false, 12288>(tbase + TM_P, sb + OFF_A1, sb + OFF_BB, ID_MMA1, false);
-            mma_commit(&bar_ap);
             issue_mma<8, false, 16384, true, 16384>(tbase + TM_C, sb + OFF_KQ, sb + OFF_SB, ID_KxMN, false);
             mma_commit(&bar_c);
             if (c + 1 < nchunks) { load_qkg(c + 1); pending_qkg = c + 1; }
