@@ -230,34 +230,51 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
 // 64-95, so that the products land in the TMEM lanes of the Qt rows.
 __device__ __forceinline__ int tp_row(int r) { return r < 32 ? r : r + 32; }
 
-// One warp's walk down block column J of X = (I + A)^-1 (its 8 output columns nt): for R = J+1 .. 3,
-// X_RJ = -X_RR (sum_{L=J}^{R-1} A_RL X_LJ) on warp-level bf16 tensor-core tiles with fp32 sums (bf16
-// operands here leave the output error unchanged in the chunk model).  Each X_LJ it needs is the
-// diagonal block (level 0's transposed copy) or one it has just formed, kept as a B fragment in
-// registers, so no other warp is waited for; T = X Diag(beta) entries are written as they are formed.
+// B fragment of a 16x8 (K x N) block of a row-major fp32 matrix (rows are K), rounded to bf16.
+__device__ __forceinline__ void load_b_frag_rm(const float* blk, int ld, int g, int t, uint32_t b[2]) {
+    b[0] = pack_bf16x2(blk[(2 * t) * ld + g], blk[(2 * t + 1) * ld + g]);
+    b[1] = pack_bf16x2(blk[(2 * t + 8) * ld + g], blk[(2 * t + 9) * ld + g]);
+}
+
+// One warp's walk down block column J of X = (I + A)^-1 (its 8 output columns nt), on warp-level
+// bf16 tensor-core tiles with fp32 sums.  With At_RL = X_RR A_RL (R > L >= J; independent products,
+// formed first), X_RJ = -sum_{L=J}^{R-1} At_RL X_LJ for R = J+1 .. 3, so the dependent chain is one
+// accumulation per block.  Each X_LJ it needs is the diagonal block (level 0's transposed copy) or
+// one it has just formed, kept as a B fragment in registers: no other warp is waited for.  T =
+// X Diag(beta) entries are written as they are formed.  (bf16 operands at these points leave the
+// output error unchanged in the chunk model.)
 template <int J>
 __device__ __forceinline__ void offdiag_column(const float* AF, const float* XF, const float* XT,
                                                const float* beta, uint8_t* sm, int nt, int lane) {
+    constexpr int NR = 3 - J;   // blocks below the diagonal in this column
     const int g4 = lane >> 2, t4 = lane & 3;
-    uint32_t xb[3 - J][2];   // B fragments of X_LJ, L = J .. 2
+    uint32_t at[NR][NR][4];     // A fragments of At_RL, [R - J - 1][L - J]
+#pragma unroll
+    for (int R = J + 1; R < 4; ++R) {
+        uint32_t xr[4];
+        load_a_frag(XF + (16 * R) * kLd + 16 * R, kLd, g4, t4, xr);
+#pragma unroll
+        for (int L = J; L < R; ++L) {
+            float d[2][4];
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+                uint32_t bf[2];
+                load_b_frag_rm(AF + (16 * R) * kLd + 16 * L + 8 * n, kLd, g4, t4, bf);
+                d[n][0] = d[n][1] = d[n][2] = d[n][3] = 0.f;
+                mma_16816(d[n], xr, bf);
+            }
+            afrag_of_acc(d, at[R - J - 1][L - J]);
+        }
+    }
+    uint32_t xb[NR][2];         // B fragments of X_LJ, L = J .. 2
     load_b_frag(XT + (16 * J + 8 * nt) * kLd + 16 * J, kLd, g4, t4, xb[0]);
     const int col = 16 * J + 8 * nt + 2 * t4;
     const float b0 = beta[col], b1 = beta[col + 1];
 #pragma unroll
     for (int R = J + 1; R < 4; ++R) {
-        float w[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int L = J; L < R; ++L) {
-            uint32_t af[4];
-            load_a_frag(AF + (16 * R) * kLd + 16 * L, kLd, g4, t4, af);
-            mma_16816(w, af, xb[L - J]);
-        }
-        // W as the B operand (its 16 rows are K) of X_RR W
-        const uint32_t wb[2] = {movmatrix_trans(pack_bf16x2(w[0], w[1])), movmatrix_trans(pack_bf16x2(w[2], w[3]))};
-        uint32_t ar[4];
-        load_a_frag(XF + (16 * R) * kLd + 16 * R, kLd, g4, t4, ar);
         float x[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_16816(x, ar, wb);
+#pragma unroll
+        for (int L = J; L < R; ++L) mma_16816(x, at[R - J - 1][L - J], xb[L - J]);
         *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(16 * R + g4), col, 8192)) =
             pack_bf16x2(-x[0] * b0, -x[1] * b1);
         *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(16 * R + g4 + 8), col, 8192)) =
@@ -289,7 +306,6 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __shared__ uint32_t tmem_base_s;
     __shared__ __align__(16) float s_beta[kC];
     __shared__ __align__(16) float s_gamma[2][kD];     // e^{Gam_63} per channel, by chunk parity (float2 stores)
-    __shared__ __align__(16) float s_refs[4][kD];      // Gam rows 16, 31, 48, 63
     __shared__ __align__(16) float s_qsum[4][kD];      // g summed over each 16-token quarter
     __shared__ float s_norm[2 * kC];                   // with the prologue: 1/|q_t|, then 1/|k_t|
 
@@ -439,18 +455,41 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
                 for (int i = 0; i < 16; ++i) { gam[i][0] += c0s; gam[i][1] += c1s; }
             }
-            if (tq & 1) {
-                // tokens 16 and 31 (quarter 1), 48 and 63 (quarter 3); e^{Gam_63} for the state decay
-                *reinterpret_cast<float2*>(&s_refs[2 * hq][ch0]) = make_float2(gam[0][0], gam[0][1]);
-                *reinterpret_cast<float2*>(&s_refs[2 * hq + 1][ch0]) = make_float2(gam[15][0], gam[15][1]);
-                if (hq)
-                    *reinterpret_cast<float2*>(&s_gamma[par][ch0]) =
-                        make_float2(ex2_approx_sub(gam[15][0] * kLog2e), ex2_approx_sub(gam[15][1] * kLog2e));
+            // the reference rows Gam_16, Gam_31, Gam_48, Gam_63 of this thread's channels, from the
+            // quarter sums and g of tokens 16 and 48 (each thread forms its own: no exchange)
+            float r16[2], r31[2], r48[2], r63[2];
+            {
+                const float2 s0 = *reinterpret_cast<const float2*>(&s_qsum[0][ch0]);
+                const float2 s1 = *reinterpret_cast<const float2*>(&s_qsum[1][ch0]);
+                const float2 s2 = *reinterpret_cast<const float2*>(&s_qsum[2][ch0]);
+                const float2 s3 = *reinterpret_cast<const float2*>(&s_qsum[3][ch0]);
+                auto g_at = [&](int t, float* gv) {
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_G + sw128_offset(t, ch0, 8192));
+                    gv[0] = __uint_as_float(w << 16);
+                    gv[1] = __uint_as_float(w & 0xFFFF0000u);
+                    if (kFused) { gv[0] = log_decay_from_logit(gv[0]); gv[1] = log_decay_from_logit(gv[1]); }
+                    if ((kFused || kPacked) && t >= nvalid) gv[0] = gv[1] = 0.f;
+                };
+                float g16[2], g48[2];
+                g_at(16, g16);
+                g_at(48, g48);
+                const float c2[2] = {s0.x + s1.x, s0.y + s1.y};
+                const float c3[2] = {c2[0] + s2.x, c2[1] + s2.y};
+                r16[0] = g16[0] + s0.x; r16[1] = g16[1] + s0.y;
+                r31[0] = c2[0]; r31[1] = c2[1];
+                r48[0] = g48[0] + c3[0]; r48[1] = g48[1] + c3[1];
+                r63[0] = c3[0] + s3.x; r63[1] = c3[1] + s3.y;
             }
-            // ---- P3: operand tiles (KQ may be rewritten once MMA3 of the previous chunk is done)
-            if (chunk > 0) ok = mbar_wait(&bar_c, ppar, p.timeout_ns);
-            ok = named_bar_and(kBarPrep, kPrepThreads, ok);
-            if (!ok) break;
+            if (tq == 3)   // e^{Gam_63} for the state decay
+                *reinterpret_cast<float2*>(&s_gamma[par][ch0]) =
+                    make_float2(ex2_approx_sub(r63[0] * kLog2e), ex2_approx_sub(r63[1] * kLog2e));
+            // ---- P3: operand tiles (KQ may be rewritten once MMA3 of the previous chunk is done;
+            // every thread waits for that itself, the vote is at the next barrier)
+            if (chunk > 0 && ok) ok = mbar_wait(&bar_c, ppar, p.timeout_ns);
+            if (kFused) {   // the inverse norms are read below
+                ok = named_bar_and(kBarPrep, kPrepThreads, ok);
+                if (!ok) break;
+            }
             uint32_t kb[16];  // Kb of these tokens, written once the previous chunk released the tile
             {
                 // per channel, against the block's reference token m: Gam_m*log2e, e^{Gam_63-Gam_m},
@@ -459,12 +498,10 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 // tokens, so at g >= -5 it stays a normal float.
                 float gmL[2], ce[2], em[2], f1[2] = {0.f, 0.f}, f2[2] = {0.f, 0.f};
                 {
-                    const float2 r16 = *reinterpret_cast<const float2*>(&s_refs[0][ch0]);
-                    const float2 r31 = *reinterpret_cast<const float2*>(&s_refs[1][ch0]);
-                    const float2 r48 = *reinterpret_cast<const float2*>(&s_refs[2][ch0]);
-                    const float2 r63 = *reinterpret_cast<const float2*>(&s_refs[3][ch0]);
-                    const float g16[2] = {r16.x, r16.y}, g31[2] = {r31.x, r31.y};
-                    const float g48[2] = {r48.x, r48.y}, g63[2] = {r63.x, r63.y};
+                    const float* g16 = r16;
+                    const float* g31 = r31;
+                    const float* g48 = r48;
+                    const float* g63 = r63;
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const float gm = hq ? g48[u] : g16[u];
@@ -516,15 +553,16 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
-            named_bar_sync(kBarPrep, kPrepThreads);
-            // KQ of this chunk is ready and its raw q, k, g consumed: the recurrence group's leader
-            // issues MMA3 and the next chunk's loads
+            ok = named_bar_and(kBarPrep, kPrepThreads, ok);
+            if (!ok) break;
             // MMA1 (A and P of the chunk) straight from this group: it is on this group's path
             if (ptid == kMma1Issuer) {
                 tc_fence_after_sync();
                 issue_mma<8, false, 16384, false, 12288>(tbase + TM_P, sb + OFF_A1, sb + OFF_BB, ID_MMA1, false);
                 mma_commit(&bar_ap);
             }
+            // KQ of this chunk is ready and its raw q, k, g consumed: the recurrence group's leader
+            // issues MMA3 and the next chunk's loads
             if (ptid == kIssuer && !(p.skip_handoff && chunk == 0)) mbar_arrive(&bar_kq);
             // ---- P4: Kb tile, P and A from TMEM, triangular solve, T tile
             if (chunk > 0) ok = mbar_wait(&bar_os, ppar, p.timeout_ns);  // T, P, Kb released

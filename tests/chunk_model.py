@@ -51,9 +51,8 @@ def kernel_inverse(A, rnd):
     """(I + A)^-1 for a strictly lower 64x64 A the way the tensor-core kernel forms it.
 
     Diagonal 16x16 blocks: N = A_bb is nilpotent, (I + N)^-1 = (I - N)(I + N^2)(I + N^4)(I + N^8),
-    every product with operands rounded by `rnd` and exact sums.  Off-diagonal blocks by block
-    distance: X_RJ = -X_RR (sum_{L=J}^{R-1} A_RL X_LJ), operands rounded, the inner sum rounded
-    once more before the outer product.
+    every product with operands rounded by `rnd` and exact sums.  Off-diagonal blocks: At_RL =
+    X_RR A_RL, then X_RJ = -sum_{L=J}^{R-1} At_RL X_LJ down each block column, operands rounded.
     """
     n = A.shape[0]
     nb = n // 16
@@ -68,12 +67,16 @@ def kernel_inverse(A, rnd):
             Np = rnd(Np) @ rnd(Np)
             P = P + rnd(P) @ rnd(Np)
         X[s, s] = P
-    for d in range(1, nb):
-        for J in range(nb - d):
-            R = J + d
-            rs, js = slice(16 * R, 16 * R + 16), slice(16 * J, 16 * J + 16)
-            W = sum(rnd(A[rs, 16 * L:16 * L + 16]) @ rnd(X[16 * L:16 * L + 16, js]) for L in range(J, R))
-            X[rs, js] = -(rnd(X[rs, rs]) @ rnd(W))
+    # off-diagonal blocks: At_RL = X_RR A_RL first (operands rounded, result rounded as the next
+    # product's operand), then X_RJ = -sum_{L=J}^{R-1} At_RL X_LJ down each block column
+    At = {}
+    for R in range(nb):
+        for L in range(R):
+            At[(R, L)] = rnd(rnd(X[16 * R:16 * R + 16, 16 * R:16 * R + 16]) @ rnd(A[16 * R:16 * R + 16, 16 * L:16 * L + 16]))
+    for J in range(nb):
+        js = slice(16 * J, 16 * J + 16)
+        for R in range(J + 1, nb):
+            X[16 * R:16 * R + 16, js] = -sum(At[(R, L)] @ rnd(X[16 * L:16 * L + 16, js]) for L in range(J, R))
     return X
 
 
