@@ -533,12 +533,22 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     const float E0 = ex2_approx(x0), E1 = ex2_approx(x1);
                     const float I0 = ex2_approx(-x0), I1 = ex2_approx(-x1);
                     const float kI0 = k0 * I0, kI1 = k1 * I1;
-                    const uint32_t a1q = pack_bf16x2(q0 * E0, q1 * E1);
-                    const uint32_t a1k = pack_bf16x2(k0 * E0, k1 * E1);
-                    // MMA1 operands: A rows [Qt0;Kt0;Qt1;Kt1], B rows [Kh0(16);Kh1(48);Kh0(48)]
+                    // MMA1 operands: A rows [Qt0;Kt0;Qt1;Kt1], B rows [Kh0(16);Kh1(48);Kh0(48)].  Without
+                    // the prologue q and k are bf16 already: bf16 q (k) times the bf16-rounded factor
+                    uint32_t a1q, a1k, b1;
+                    if (kFused) {
+                        a1q = pack_bf16x2(q0 * E0, q1 * E1);
+                        a1k = pack_bf16x2(k0 * E0, k1 * E1);
+                        b1 = pack_bf16x2(kI0, kI1);
+                    } else {
+                        const uint32_t e2 = pack_bf16x2(E0, E1), i2 = pack_bf16x2(I0, I1);
+                        a1q = mul_bf16x2(qw, e2);
+                        a1k = mul_bf16x2(kw, e2);
+                        b1 = mul_bf16x2(kw, i2);
+                    }
                     *reinterpret_cast<uint32_t*>(sm + OFF_A1 + sw128_offset(rq, ch0, 16384)) = a1q;
                     *reinterpret_cast<uint32_t*>(sm + OFF_A1 + sw128_offset(rk, ch0, 16384)) = a1k;
-                    *reinterpret_cast<uint32_t*>(sm + OFF_BB + sw128_offset(t, ch0, 12288)) = pack_bf16x2(kI0, kI1);
+                    *reinterpret_cast<uint32_t*>(sm + OFF_BB + sw128_offset(t, ch0, 12288)) = b1;
                     // block-0 keys against token 48: k e^{Gam_16-Gam_j} e^{Gam_31-Gam_16} e^{Gam_48-Gam_31},
                     // multiplied left to right; the middle product k e^{Gam_31-Gam_j} never exceeds |k|,
                     // so a factor flushes to zero only when the exact product is below the fp32 range

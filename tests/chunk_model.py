@@ -121,9 +121,11 @@ def chunk_head(q, k, v, g, beta, S0, C=64, sub=32, bf16=False, offdiag_ref="bloc
                     ej = np.exp(ref - Gam[cols])
                 if J != R and offdiag_ref == "row_middle":
                     ej = _ftz(ej)
-                qs = rnd(qc[rows] * er)
-                ks = rnd(kc[rows] * er)
-                kh = rnd(kc[cols] * ej)
+                # the kernel multiplies the bf16 q and k by bf16-rounded factors (two roundings), except
+                # the block-1 x block-0 columns, which it forms in fp32 (one rounding)
+                qs = rnd(qc[rows] * rnd(er))
+                ks = rnd(kc[rows] * rnd(er))
+                kh = rnd(kc[cols] * ej) if J != R else rnd(kc[cols] * rnd(ej))
                 P[rows, cols] = qs @ kh.T
                 A[rows, cols] = ks @ kh.T
         with np.errstate(invalid="ignore", over="ignore"):
@@ -138,8 +140,8 @@ def chunk_head(q, k, v, g, beta, S0, C=64, sub=32, bf16=False, offdiag_ref="bloc
             # bf16 e^{Gam_ref}: two roundings
             refs = np.repeat(Gam[sub // 2::sub], sub, axis=0)
             with np.errstate(over="ignore"):
-                Kt = rnd(rnd(kc * np.exp(Gam - refs)) * rnd(np.exp(refs)))
-                Qt = rnd(rnd(qc * np.exp(Gam - refs)) * rnd(np.exp(refs)))
+                Kt = rnd(rnd(kc * rnd(np.exp(Gam - refs))) * rnd(np.exp(refs)))
+                Qt = rnd(rnd(qc * rnd(np.exp(Gam - refs))) * rnd(np.exp(refs)))
         else:
             Kt = kc * np.exp(Gam)
             Qt = qc * np.exp(Gam)
