@@ -64,12 +64,14 @@ constexpr uint32_t OFF_V = 49152;           // v, then Y = V - Kt S, then U (MN-
 constexpr uint32_t OFF_AP = 65536;          // prep operand region (56 KB)
 constexpr uint32_t OFF_A1 = OFF_AP;                 // [Qt0;Kt0;Qt1;Kt1] block-middle refs, K-major, 2 x 16 KB
 constexpr uint32_t OFF_BB = OFF_AP + 32768;         // [Kh0(16);Kh1(48);Kh0(48)], K-major, 96 rows, 2 x 12 KB
-constexpr int kLd = 68;                              // padded row stride (floats) of the solve matrices
-constexpr int kLdS = 20;
-constexpr uint32_t OFF_AF = OFF_AP;                  // after MMA1: A (fp32 64 x kLd)
-constexpr uint32_t OFF_X = OFF_AF + 64 * kLd * 4;    //   X = (I+A)^-1, row-major
-constexpr uint32_t OFF_XT = OFF_X + 64 * kLd * 4;    //   X transposed
-constexpr uint32_t OFF_WS = OFF_XT + 64 * kLd * 4;   //   per-warp W^T scratch (8 warps x 8 x kLdS)
+// The solve's scratch, in the MMA1 B-operand space (free once MMA1 is done; the A-operand space is
+// left alone): the diagonal 16x16 blocks of A in fp32 (padded rows of kLdD floats), A in bf16
+// (row-major, rows of kLdA elements) for the off-diagonal blocks, and the diagonal blocks of
+// X = (I+A)^-1 in bf16 (rows of kLdX elements).  bf16 rows are 16-byte aligned for ldmatrix.
+constexpr int kLdD = 20, kLdA = 72, kLdX = 24;
+constexpr uint32_t OFF_AFD = OFF_BB;
+constexpr uint32_t OFF_AOFF = OFF_AFD + 4 * 16 * kLdD * 4;
+constexpr uint32_t OFF_XD = OFF_AOFF + 64 * kLdA * 2;
 constexpr uint32_t OFF_KQ = OFF_AP + 57344;          // [Qt0;Kt0;Qt1;Kt1] chunk-start ref, K-major, 2 x 16 KB
 constexpr uint32_t OFF_SB = OFF_KQ + 32768;          // S in bf16, MN-major B (K = dk), 2 x 16 KB
 constexpr uint32_t OFF_TP = OFF_SB + 32768;          // T and P, interleaved 4 KB pieces (16 KB)
@@ -78,7 +80,7 @@ constexpr uint32_t OFF_P = OFF_TP + 4096;            //   P rows 0-31 at +4 KB, 
 constexpr uint32_t OFF_KBAR = OFF_TP + 16384;        // Kb, MN-major A (M = dk), 2 x 8 KB
 constexpr uint32_t SMEM_BYTES = OFF_KBAR + 16384;    // 221184
 constexpr uint32_t SMEM_DYN = SMEM_BYTES + 1024;     // + alignment slack
-static_assert(OFF_WS + 8 * 8 * kLdS * 4 <= OFF_KQ, "solve scratch overlaps KQ");
+static_assert(OFF_XD + 4 * 16 * kLdX * 2 <= OFF_BB + 2 * 12288, "solve scratch leaves the MMA1 B space");
 static_assert(OFF_BB + 2 * 12288 <= OFF_KQ, "BB overlaps KQ");
 
 // ---- TMEM columns (fp32 accumulators, 128 lanes) ----
@@ -149,21 +151,6 @@ __device__ __forceinline__ void mma_16816(float d[4], const uint32_t a[4], const
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
-// A fragment from a row-major fp32 16x16 block (row stride ld floats), rounded to bf16.
-__device__ __forceinline__ void load_a_frag(const float* blk, int ld, int g, int t, uint32_t a[4]) {
-    const float2 v0 = *reinterpret_cast<const float2*>(blk + g * ld + 2 * t);
-    const float2 v1 = *reinterpret_cast<const float2*>(blk + (g + 8) * ld + 2 * t);
-    const float2 v2 = *reinterpret_cast<const float2*>(blk + g * ld + 2 * t + 8);
-    const float2 v3 = *reinterpret_cast<const float2*>(blk + (g + 8) * ld + 2 * t + 8);
-    a[0] = pack_bf16x2(v0.x, v0.y); a[1] = pack_bf16x2(v1.x, v1.y);
-    a[2] = pack_bf16x2(v2.x, v2.y); a[3] = pack_bf16x2(v3.x, v3.y);
-}
-// B fragment of a 16x8 (K x N) block stored transposed (row n holds the 16 K values), rounded to bf16.
-__device__ __forceinline__ void load_b_frag(const float* blkT, int ld, int g, int t, uint32_t b[2]) {
-    const float2 v0 = *reinterpret_cast<const float2*>(blkT + g * ld + 2 * t);
-    const float2 v1 = *reinterpret_cast<const float2*>(blkT + g * ld + 2 * t + 8);
-    b[0] = pack_bf16x2(v0.x, v0.y); b[1] = pack_bf16x2(v1.x, v1.y);
-}
 
 // 8x8 transpose of b16 pairs across the warp (thread i holds row i/4, columns 2(i%4) and 2(i%4)+1).
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
@@ -230,11 +217,21 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
 // 64-95, so that the products land in the TMEM lanes of the Qt rows.
 __device__ __forceinline__ int tp_row(int r) { return r < 32 ? r : r + 32; }
 
-// B fragment of a 16x8 (K x N) block of a row-major fp32 matrix (rows are K), rounded to bf16.
-__device__ __forceinline__ void load_b_frag_rm(const float* blk, int ld, int g, int t, uint32_t b[2]) {
-    b[0] = pack_bf16x2(blk[(2 * t) * ld + g], blk[(2 * t + 1) * ld + g]);
-    b[1] = pack_bf16x2(blk[(2 * t + 8) * ld + g], blk[(2 * t + 9) * ld + g]);
+// Fragments from bf16 tiles in shared memory (row addresses 16-byte aligned): the A fragment of a
+// 16x16 row-major block, and the B fragment of a 16x8 (K x N) block of a row-major (K rows) matrix.
+__device__ __forceinline__ void ldsm_a16(uint32_t base, uint32_t row_bytes, int lane, uint32_t a[4]) {
+    const uint32_t m = lane >> 3, rr = lane & 7;
+    const uint32_t addr = base + (rr + 8 * (m & 1)) * row_bytes + 16 * (m >> 1);
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]) : "r"(addr) : "memory");
 }
+__device__ __forceinline__ void ldsm_b16x8_trans(uint32_t base, uint32_t row_bytes, int lane, uint32_t b[2]) {
+    const uint32_t rr = lane & 15;   // lanes 16-31 repeat 0-15 (their addresses are not used)
+    const uint32_t addr = base + rr * row_bytes;
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+                 : "=r"(b[0]), "=r"(b[1]) : "r"(addr) : "memory");
+}
+
 
 // One warp's walk down block column J of X = (I + A)^-1 (its 8 output columns nt), on warp-level
 // bf16 tensor-core tiles with fp32 sums.  With At_RL = X_RR A_RL (R > L >= J; independent products,
@@ -244,22 +241,21 @@ __device__ __forceinline__ void load_b_frag_rm(const float* blk, int ld, int g, 
 // X Diag(beta) entries are written as they are formed.  (bf16 operands at these points leave the
 // output error unchanged in the chunk model.)
 template <int J>
-__device__ __forceinline__ void offdiag_column(const float* AF, const float* XF, const float* XT,
-                                               const float* beta, uint8_t* sm, int nt, int lane) {
+__device__ __forceinline__ void offdiag_column(uint32_t sb, const float* beta, uint8_t* sm, int nt, int lane) {
     constexpr int NR = 3 - J;   // blocks below the diagonal in this column
     const int g4 = lane >> 2, t4 = lane & 3;
     uint32_t at[NR][NR][4];     // A fragments of At_RL, [R - J - 1][L - J]
 #pragma unroll
     for (int R = J + 1; R < 4; ++R) {
         uint32_t xr[4];
-        load_a_frag(XF + (16 * R) * kLd + 16 * R, kLd, g4, t4, xr);
+        ldsm_a16(sb + OFF_XD + 16 * R * kLdX * 2, kLdX * 2, lane, xr);
 #pragma unroll
         for (int L = J; L < R; ++L) {
             float d[2][4];
 #pragma unroll
             for (int n = 0; n < 2; ++n) {
                 uint32_t bf[2];
-                load_b_frag_rm(AF + (16 * R) * kLd + 16 * L + 8 * n, kLd, g4, t4, bf);
+                ldsm_b16x8_trans(sb + OFF_AOFF + (16 * R) * kLdA * 2 + (16 * L + 8 * n) * 2, kLdA * 2, lane, bf);
                 d[n][0] = d[n][1] = d[n][2] = d[n][3] = 0.f;
                 mma_16816(d[n], xr, bf);
             }
@@ -267,7 +263,7 @@ __device__ __forceinline__ void offdiag_column(const float* AF, const float* XF,
         }
     }
     uint32_t xb[NR][2];         // B fragments of X_LJ, L = J .. 2
-    load_b_frag(XT + (16 * J + 8 * nt) * kLd + 16 * J, kLd, g4, t4, xb[0]);
+    ldsm_b16x8_trans(sb + OFF_XD + 16 * J * kLdX * 2 + 8 * nt * 2, kLdX * 2, lane, xb[0]);
     const int col = 16 * J + 8 * nt + 2 * t4;
     const float b0 = beta[col], b1 = beta[col + 1];
 #pragma unroll
@@ -375,9 +371,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         for (int idx = ptid; idx < 512; idx += kPrepThreads)
             *reinterpret_cast<uint4*>(sm + OFF_T + sw128_offset(tp_row(idx >> 3), (idx & 7) * 8, 8192)) =
                 make_uint4(0u, 0u, 0u, 0u);
-        float* AF = reinterpret_cast<float*>(sm + OFF_AF);
-        float* XF = reinterpret_cast<float*>(sm + OFF_X);
-        float* XT = reinterpret_cast<float*>(sm + OFF_XT);
+        float* AFD = reinterpret_cast<float*>(sm + OFF_AFD);
         // this thread's part of the Gam scan and of the element-wise step: channels ch0, ch0 + 1 of the
         // 16 tokens of quarter tq (a warp covers 64 channels of one quarter)
         const int tq = warp >> 1;
@@ -617,16 +611,23 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         *reinterpret_cast<uint4*>(sm + OFF_P + sw128_offset(tp_row(r), jb + j, 8192)) = pack8(v8);
                     }
                 } else {
-                    // A row r: strictly lower, scaled by beta_r (select first: masked entries may be inf)
+                    // A row r: strictly lower, scaled by beta_r (select first: masked entries may be inf),
+                    // in bf16; the diagonal block's 16 entries also in fp32 (quarter 1 with columns
+                    // 0-31 and quarter 3 with columns 32-63 hold the diagonal blocks)
                     const float br = s_beta[r];
+                    float w[32];
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        float4 w4;
-                        w4.x = (jb + j + 0 < r) ? br * row[j + 0] : 0.f;
-                        w4.y = (jb + j + 1 < r) ? br * row[j + 1] : 0.f;
-                        w4.z = (jb + j + 2 < r) ? br * row[j + 2] : 0.f;
-                        w4.w = (jb + j + 3 < r) ? br * row[j + 3] : 0.f;
-                        *reinterpret_cast<float4*>(AF + r * kLd + jb + j) = w4;
+                    for (int j = 0; j < 32; ++j) w[j] = (jb + j < r) ? br * row[j] : 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8)
+                        *reinterpret_cast<uint4*>(sm + OFF_AOFF + r * kLdA * 2 + (jb + j) * 2) = pack8(w + j);
+                    if ((quarter == 1 && colhalf == 0) || (quarter == 3 && colhalf == 1)) {
+                        const bool hi = (r & 16) != 0;    // the row's diagonal block is columns 16-31 of the 32
+                        float* dst = AFD + ((r >> 4) * 16 + (r & 15)) * kLdD;
+#pragma unroll
+                        for (int j = 0; j < 16; j += 4)
+                            *reinterpret_cast<float4*>(dst + j) = make_float4(hi ? w[16 + j] : w[j], hi ? w[17 + j] : w[j + 1],
+                                                                              hi ? w[18 + j] : w[j + 2], hi ? w[19 + j] : w[j + 3]);
                     }
                 }
             }
@@ -644,7 +645,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
                     for (int hr = 0; hr < 2; ++hr) {
                         const int row = g4 + 8 * hr, col = 8 * nt + 2 * t4;
-                        const float2 v = *reinterpret_cast<const float2*>(AF + (o0 + row) * kLd + o0 + col);
+                        const float2 v = *reinterpret_cast<const float2*>(AFD + (o0 + row) * kLdD + col);
                         nn[nt][2 * hr] = v.x;
                         nn[nt][2 * hr + 1] = v.y;
                         xm[nt][2 * hr] = (row == col ? 1.f : 0.f) - v.x;
@@ -663,7 +664,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
                         for (int e = 0; e < 4; ++e) nn[nt][e] = sq[nt][e];
                 }
-                // X, X^T (fp32, for the off-diagonal levels) and T = X Diag(beta) (bf16)
+                // X (bf16, for the off-diagonal blocks) and T = X Diag(beta) (bf16)
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
                     const int col = 8 * nt + 2 * t4;
@@ -672,9 +673,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     for (int hr = 0; hr < 2; ++hr) {
                         const int row = g4 + 8 * hr;
                         const float x0 = xm[nt][2 * hr], x1 = xm[nt][2 * hr + 1];
-                        *reinterpret_cast<float2*>(XF + (o0 + row) * kLd + o0 + col) = make_float2(x0, x1);
-                        XT[(o0 + col) * kLd + o0 + row] = x0;
-                        XT[(o0 + col + 1) * kLd + o0 + row] = x1;
+                        *reinterpret_cast<uint32_t*>(sm + OFF_XD + ((o0 + row) * kLdX + col) * 2) = pack_bf16x2(x0, x1);
                         *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(o0 + row), o0 + col, 8192)) =
                             pack_bf16x2(x0 * b0, x1 * b1);
                     }
@@ -684,9 +683,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // off-diagonal blocks, one block column per warp pair (8 output columns per warp)
             if (warp < 6) {
                 const int nt = warp & 1;
-                if (warp < 2) offdiag_column<0>(AF, XF, XT, s_beta, sm, nt, lane);
-                else if (warp < 4) offdiag_column<1>(AF, XF, XT, s_beta, sm, nt, lane);
-                else offdiag_column<2>(AF, XF, XT, s_beta, sm, nt, lane);
+                if (warp < 2) offdiag_column<0>(sb, s_beta, sm, nt, lane);
+                else if (warp < 4) offdiag_column<1>(sb, s_beta, sm, nt, lane);
+                else offdiag_column<2>(sb, s_beta, sm, nt, lane);
             }
             fence_proxy_async_smem();
             named_bar_sync(kBarPrep, kPrepThreads);
