@@ -297,12 +297,13 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t sb = smem_u32(sm);
 
     // TMA / MMA completion barriers (one phase per chunk) and prep -> serial hand-offs.
-    __shared__ uint64_t bar_qkg, bar_v, bar_ap, bar_c, bar_u, bar_os, bar_kq, bar_tpk;
+    __shared__ uint64_t bar_qk, bar_g, bar_v, bar_ap, bar_c, bar_u, bar_os, bar_kq, bar_tpk;
     __shared__ uint64_t bar_drain_p, bar_drain_s, bar_drain_g;
     __shared__ uint32_t tmem_base_s;
     __shared__ __align__(16) float s_beta[kC];
     __shared__ __align__(16) float s_gamma[2][kD];     // e^{Gam_63} per channel, by chunk parity (float2 stores)
     __shared__ __align__(16) float s_qsum[4][kD];      // g summed over each 16-token quarter
+    __shared__ __align__(16) float s_g1648[2][kD];     // g of tokens 16 and 48 (raw g is dead after the scan)
     __shared__ float s_norm[2 * kC];                   // with the prologue: 1/|q_t|, then 1/|k_t|
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -329,7 +330,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const int nchunks = (T + kC - 1) / kC;
 
     if (tid == 0) {
-        mbar_init(&bar_qkg, 1); mbar_init(&bar_v, 1); mbar_init(&bar_ap, 1);
+        mbar_init(&bar_qk, 1); mbar_init(&bar_g, 1); mbar_init(&bar_v, 1); mbar_init(&bar_ap, 1);
         mbar_init(&bar_c, 1); mbar_init(&bar_u, 1); mbar_init(&bar_os, 1); mbar_init(&bar_kq, 1);
         mbar_init(&bar_tpk, 1); mbar_init(&bar_drain_p, 1); mbar_init(&bar_drain_s, 1); mbar_init(&bar_drain_g, 1);
         fence_mbar_init();
@@ -346,14 +347,21 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t tbase = tmem_base_s;
     const uint32_t tlane = tbase + ((uint32_t)(32 * quarter) << 16);  // this warp's lane quarter
 
-    auto load_qkg = [&](int chunk) {
-        mbar_arrive_expect_tx(&bar_qkg, 3u * 16384u);
+    // raw q and k are read until the chunk's operand tiles are written; raw g only by the scan,
+    // so the next chunk's g is loaded a step earlier than its q and k
+    auto load_qk = [&](int chunk) {
+        mbar_arrive_expect_tx(&bar_qk, 2u * 16384u);
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-            tma_load_4d(sm + OFF_RAW_Q + x * 8192, &tm_q, &bar_qkg, 64 * x, h, tok0 + chunk * kC, bmap);
-            tma_load_4d(sm + OFF_RAW_K + x * 8192, &tm_k, &bar_qkg, 64 * x, h, tok0 + chunk * kC, bmap);
-            tma_load_4d(sm + OFF_RAW_G + x * 8192, &tm_g, &bar_qkg, 64 * x, h, tok0 + chunk * kC, bmap);
+            tma_load_4d(sm + OFF_RAW_Q + x * 8192, &tm_q, &bar_qk, 64 * x, h, tok0 + chunk * kC, bmap);
+            tma_load_4d(sm + OFF_RAW_K + x * 8192, &tm_k, &bar_qk, 64 * x, h, tok0 + chunk * kC, bmap);
         }
+    };
+    auto load_g = [&](int chunk) {
+        mbar_arrive_expect_tx(&bar_g, 16384u);
+#pragma unroll
+        for (int x = 0; x < 2; ++x)
+            tma_load_4d(sm + OFF_RAW_G + x * 8192, &tm_g, &bar_g, 64 * x, h, tok0 + chunk * kC, bmap);
     };
     auto load_v = [&](int chunk) {
         mbar_arrive_expect_tx(&bar_v, 16384u);
@@ -365,8 +373,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (is_prep) {
         // ====================================================================== prep group
         const int ptid = tid;                               // 0..255
-        int pending = -1;                                   // chunk whose q,k,g loads are in flight (issuer)
-        if (ptid == kIssuer) { load_qkg(0); pending = 0; }
+        int pending_g = -1, pending_qk = -1;                // chunks whose g / q,k loads this issuer has in flight
+        if (ptid == kIssuer) { load_g(0); load_qk(0); pending_g = 0; pending_qk = 0; }
         // T's strictly upper 16x16 blocks stay zero for the whole sequence: clear the tile once
         for (int idx = ptid; idx < 512; idx += kPrepThreads)
             *reinterpret_cast<uint4*>(sm + OFF_T + sw128_offset(tp_row(idx >> 3), (idx & 7) * 8, 8192)) =
@@ -394,8 +402,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 s_beta[ptid] = kFused ? (chunk * kC + ptid < T ? sigmoid_fast(bz) : 0.f) : bz;
             }
             if (chunk + 1 < nchunks) beta_next = fetch_beta(chunk + 1);
-            ok = mbar_wait(&bar_qkg, par, p.timeout_ns);   // every thread: its own view of the TMA data
-            if (ok && ptid == kIssuer) pending = -1;
+            ok = mbar_wait(&bar_g, par, p.timeout_ns);     // every thread: its own view of the TMA data
+            if (ok && ptid == kIssuer) pending_g = -1;
             // ---- P2: Gam = in-chunk prefix sum of g in fp32: the running sum over this quarter,
             // then the totals of the quarters before it
             // rows past nvalid are padding: the tensor map reads zeros there for the [B, T, H, d] layout,
@@ -416,9 +424,17 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     gam[i][1] = a1;
                 }
                 *reinterpret_cast<float2*>(&s_qsum[tq][ch0]) = make_float2(a0, a1);
+                if (tq & 1)   // the first token of quarter 1 (3) is token 16 (48): its sum is its g
+                    *reinterpret_cast<float2*>(&s_g1648[tq >> 1][ch0]) = make_float2(gam[0][0], gam[0][1]);
             }
             ok = named_bar_and(kBarPrep, kPrepThreads, ok);
             if (!ok) break;
+            // raw g of this chunk is consumed: load the next chunk's
+            if (ptid == kIssuer && chunk + 1 < nchunks) { load_g(chunk + 1); pending_g = chunk + 1; }
+            if (kFused) {   // the norms below read raw q and k
+                ok = mbar_wait(&bar_qk, par, p.timeout_ns);
+                if (ok && ptid == kIssuer) pending_qk = -1;
+            }
             if (kFused) {
                 // 1/|x| of every q and k row of the chunk (row = thread/2, 64 channels per thread)
                 const int row = ptid >> 1, half = ptid & 1, t = row & (kC - 1);
@@ -457,16 +473,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const float2 s1 = *reinterpret_cast<const float2*>(&s_qsum[1][ch0]);
                 const float2 s2 = *reinterpret_cast<const float2*>(&s_qsum[2][ch0]);
                 const float2 s3 = *reinterpret_cast<const float2*>(&s_qsum[3][ch0]);
-                auto g_at = [&](int t, float* gv) {
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_G + sw128_offset(t, ch0, 8192));
-                    gv[0] = __uint_as_float(w << 16);
-                    gv[1] = __uint_as_float(w & 0xFFFF0000u);
-                    if (kFused) { gv[0] = log_decay_from_logit(gv[0]); gv[1] = log_decay_from_logit(gv[1]); }
-                    if ((kFused || kPacked) && t >= nvalid) gv[0] = gv[1] = 0.f;
-                };
-                float g16[2], g48[2];
-                g_at(16, g16);
-                g_at(48, g48);
+                const float2 g16v = *reinterpret_cast<const float2*>(&s_g1648[0][ch0]);
+                const float2 g48v = *reinterpret_cast<const float2*>(&s_g1648[1][ch0]);
+                const float g16[2] = {g16v.x, g16v.y}, g48[2] = {g48v.x, g48v.y};
                 const float c2[2] = {s0.x + s1.x, s0.y + s1.y};
                 const float c3[2] = {c2[0] + s2.x, c2[1] + s2.y};
                 r16[0] = g16[0] + s0.x; r16[1] = g16[1] + s0.y;
@@ -479,6 +488,10 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     make_float2(ex2_approx_sub(r63[0] * kLog2e), ex2_approx_sub(r63[1] * kLog2e));
             // ---- P3: operand tiles (KQ may be rewritten once MMA3 of the previous chunk is done;
             // every thread waits for that itself, the vote is at the next barrier)
+            if (!kFused && ok) {
+                ok = mbar_wait(&bar_qk, par, p.timeout_ns);
+                if (ok && ptid == kIssuer) pending_qk = -1;
+            }
             if (chunk > 0 && ok) ok = mbar_wait(&bar_c, ppar, p.timeout_ns);
             if (kFused) {   // the inverse norms are read below
                 ok = named_bar_and(kBarPrep, kPrepThreads, ok);
@@ -700,20 +713,21 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (ptid == kIssuer) {
             mma_commit(&bar_drain_p);
             if (!mbar_wait(&bar_drain_p, 0, p.timeout_ns)) report_status(p.status, KDA_ERR_TIMEOUT);
-            if (pending >= 0) (void)mbar_wait(&bar_qkg, (uint32_t)(pending & 1), p.timeout_ns);
+            if (pending_g >= 0) (void)mbar_wait(&bar_g, (uint32_t)(pending_g & 1), p.timeout_ns);
+            if (pending_qk >= 0) (void)mbar_wait(&bar_qk, (uint32_t)(pending_qk & 1), p.timeout_ns);
         }
     } else {
         // ====================================================================== serial group
         const int stid = tid - kPrepThreads;                // 0..255
         int pending = -1;                                   // chunk whose v load is in flight
-        int pending_qkg = -1;                               // last chunk whose q,k,g loads this leader issued
+        int pending_qk = -1;                                // last chunk whose q,k loads this leader issued
         // Once the prep group has published chunk c's operand tiles (bar_kq): MMA3 = [Qt0;Kt0;Qt1;Kt1] S
         // and the raw q, k, g of chunk c+1 into the buffers the prep group has finished reading.
         auto issue_for_chunk = [&](int c) {
             tc_fence_after_sync();
             issue_mma<8, false, 16384, true, 16384>(tbase + TM_C, sb + OFF_KQ, sb + OFF_SB, ID_KxMN, false);
             mma_commit(&bar_c);
-            if (c + 1 < nchunks) { load_qkg(c + 1); pending_qkg = c + 1; }
+            if (c + 1 < nchunks) { load_qk(c + 1); pending_qk = c + 1; }
         };
         // initial state: fp32 into TMEM, bf16 copy into the MN-major S tile
         {
@@ -890,7 +904,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mma_commit(&bar_drain_s);
             if (!mbar_wait(&bar_drain_s, 0, p.timeout_ns)) report_status(p.status, KDA_ERR_TIMEOUT);
             if (pending >= 0) (void)mbar_wait(&bar_v, (uint32_t)(pending & 1), p.timeout_ns);
-            if (pending_qkg >= 0) (void)mbar_wait(&bar_qkg, (uint32_t)(pending_qkg & 1), p.timeout_ns);
+            if (pending_qk >= 0) (void)mbar_wait(&bar_qk, (uint32_t)(pending_qk & 1), p.timeout_ns);
         }
         named_bar_sync(kBarSerial, kSerialThreads);
         tc_fence_after_sync();
