@@ -119,6 +119,37 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&p);
 }
+__device__ __forceinline__ uint32_t pack_bf16x2(float2 v) { return pack_bf16x2(v.x, v.y); }
+// Two fp32 lanes in one instruction (sm_100 f32x2 arithmetic; each lane is rounded as the
+// scalar operation rounds it, so results are those of the scalar code)
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
 
 // Byte offset of K step kk (16 elements) inside an operand tile: K-major tiles advance 32 B
 // inside a 128-byte swizzle row and jump to the next 64-column atom every 4 steps; MN-major
@@ -272,9 +303,9 @@ __device__ __forceinline__ void offdiag_column(uint32_t sb, const float* beta, u
 #pragma unroll
         for (int L = J; L < R; ++L) mma_16816(x, at[R - J - 1][L - J], xb[L - J]);
         *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(16 * R + g4), col, 8192)) =
-            pack_bf16x2(-x[0] * b0, -x[1] * b1);
+            pack_bf16x2(mul2(make_float2(-x[0], -x[1]), make_float2(b0, b1)));
         *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(16 * R + g4 + 8), col, 8192)) =
-            pack_bf16x2(-x[2] * b0, -x[3] * b1);
+            pack_bf16x2(mul2(make_float2(-x[2], -x[3]), make_float2(b0, b1)));
         if (R < 3) {
             xb[R - J][0] = movmatrix_trans(pack_bf16x2(-x[0], -x[1]));
             xb[R - J][1] = movmatrix_trans(pack_bf16x2(-x[2], -x[3]));
@@ -409,23 +440,21 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // rows past nvalid are padding: the tensor map reads zeros there for the [B, T, H, d] layout,
             // but the next sequence's rows for packed sequences, and a zero logit is no zero gate
             const int nvalid = min(kC, T - chunk * kC);
-            float gam[16][2];
+            float2 gam[16];
             {
-                float a0 = 0.f, a1 = 0.f;
+                float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const uint32_t w = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_G + sw128_offset(16 * tq + i, ch0, 8192));
                     float g0 = __uint_as_float(w << 16), g1 = __uint_as_float(w & 0xFFFF0000u);
                     if (kFused) { g0 = log_decay_from_logit(g0); g1 = log_decay_from_logit(g1); }
                     if ((kFused || kPacked) && 16 * tq + i >= nvalid) g0 = g1 = 0.f;
-                    a0 += g0;
-                    a1 += g1;
-                    gam[i][0] = a0;
-                    gam[i][1] = a1;
+                    acc = add2(acc, make_float2(g0, g1));
+                    gam[i] = acc;
                 }
-                *reinterpret_cast<float2*>(&s_qsum[tq][ch0]) = make_float2(a0, a1);
+                *reinterpret_cast<float2*>(&s_qsum[tq][ch0]) = acc;
                 if (tq & 1)   // the first token of quarter 1 (3) is token 16 (48): its sum is its g
-                    *reinterpret_cast<float2*>(&s_g1648[tq >> 1][ch0]) = make_float2(gam[0][0], gam[0][1]);
+                    *reinterpret_cast<float2*>(&s_g1648[tq >> 1][ch0]) = gam[0];
             }
             ok = named_bar_and(kBarPrep, kPrepThreads, ok);
             if (!ok) break;
@@ -439,31 +468,27 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 // 1/|x| of every q and k row of the chunk (row = thread/2, 64 channels per thread)
                 const int row = ptid >> 1, half = ptid & 1, t = row & (kC - 1);
                 const uint8_t* tile = sm + (row < kC ? OFF_RAW_Q : OFF_RAW_K) + half * 8192 + t * 128;
-                float ss = 0.f;
+                float2 ss2 = make_float2(0.f, 0.f);   // even and odd channels
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const uint4 w4 = *reinterpret_cast<const uint4*>(tile + ((j ^ (t & 7)) << 4));
                     const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float lo = __uint_as_float(wv[e] << 16), hi = __uint_as_float(wv[e] & 0xFFFF0000u);
-                        ss = fmaf(lo, lo, ss);
-                        ss = fmaf(hi, hi, ss);
+                        const float2 x2 = make_float2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
+                        ss2 = fma2(x2, x2, ss2);
                     }
                 }
+                float ss = ss2.x + ss2.y;
                 ss += __shfl_xor_sync(0xffffffffu, ss, 1);
                 if (half == 0) s_norm[row] = ss > 0.f ? rsqrtf(ss) : 0.f;
             }
             {
-                float c0s = 0.f, c1s = 0.f;
+                float2 carry = make_float2(0.f, 0.f);
 #pragma unroll 1
-                for (int qq = 0; qq < tq; ++qq) {
-                    const float2 s2 = *reinterpret_cast<const float2*>(&s_qsum[qq][ch0]);
-                    c0s += s2.x;
-                    c1s += s2.y;
-                }
+                for (int qq = 0; qq < tq; ++qq) carry = add2(carry, *reinterpret_cast<const float2*>(&s_qsum[qq][ch0]));
 #pragma unroll
-                for (int i = 0; i < 16; ++i) { gam[i][0] += c0s; gam[i][1] += c1s; }
+                for (int i = 0; i < 16; ++i) gam[i] = add2(gam[i], carry);
             }
             // the reference rows Gam_16, Gam_31, Gam_48, Gam_63 of this thread's channels, from the
             // quarter sums and g of tokens 16 and 48 (each thread forms its own: no exchange)
@@ -475,13 +500,12 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const float2 s3 = *reinterpret_cast<const float2*>(&s_qsum[3][ch0]);
                 const float2 g16v = *reinterpret_cast<const float2*>(&s_g1648[0][ch0]);
                 const float2 g48v = *reinterpret_cast<const float2*>(&s_g1648[1][ch0]);
-                const float g16[2] = {g16v.x, g16v.y}, g48[2] = {g48v.x, g48v.y};
-                const float c2[2] = {s0.x + s1.x, s0.y + s1.y};
-                const float c3[2] = {c2[0] + s2.x, c2[1] + s2.y};
-                r16[0] = g16[0] + s0.x; r16[1] = g16[1] + s0.y;
-                r31[0] = c2[0]; r31[1] = c2[1];
-                r48[0] = g48[0] + c3[0]; r48[1] = g48[1] + c3[1];
-                r63[0] = c3[0] + s3.x; r63[1] = c3[1] + s3.y;
+                const float2 c2 = add2(s0, s1), c3 = add2(c2, s2);
+                const float2 v16 = add2(g16v, s0), v48 = add2(g48v, c3), v63 = add2(c3, s3);
+                r16[0] = v16.x; r16[1] = v16.y;
+                r31[0] = c2.x; r31[1] = c2.y;
+                r48[0] = v48.x; r48[1] = v48.y;
+                r63[0] = v63.x; r63[1] = v63.y;
             }
             if (tq == 3)   // e^{Gam_63} for the state decay
                 *reinterpret_cast<float2*>(&s_gamma[par][ch0]) =
@@ -503,23 +527,29 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 // e^{Gam_m} (bf16 pair), and for block 0 the two factors of the column change to
                 // token 48, e^{Gam_31-Gam_16} and e^{Gam_48-Gam_31}.  Each factor spans at most 17
                 // tokens, so at g >= -5 it stays a normal float.
-                float gmL[2], ce[2], em[2], f1[2] = {0.f, 0.f}, f2[2] = {0.f, 0.f};
+                float2 ngmL, ce, f1 = make_float2(0.f, 0.f), f2 = make_float2(0.f, 0.f);
+                float em[2];
                 {
                     const float* g16 = r16;
                     const float* g31 = r31;
                     const float* g48 = r48;
                     const float* g63 = r63;
+                    float gmL[2], c[2], a[2] = {0.f, 0.f}, b[2] = {0.f, 0.f};
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const float gm = hq ? g48[u] : g16[u];
                         gmL[u] = gm * kLog2e;
-                        ce[u] = ex2_approx_sub((g63[u] - gm) * kLog2e);
+                        c[u] = ex2_approx_sub((g63[u] - gm) * kLog2e);
                         em[u] = ex2_approx_sub(gm * kLog2e);
                         if (hq == 0) {
-                            f1[u] = ex2_approx_sub((g31[u] - g16[u]) * kLog2e);
-                            f2[u] = ex2_approx_sub((g48[u] - g31[u]) * kLog2e);
+                            a[u] = ex2_approx_sub((g31[u] - g16[u]) * kLog2e);
+                            b[u] = ex2_approx_sub((g48[u] - g31[u]) * kLog2e);
                         }
                     }
+                    ngmL = make_float2(-gmL[0], -gmL[1]);
+                    ce = make_float2(c[0], c[1]);
+                    f1 = make_float2(a[0], a[1]);
+                    f2 = make_float2(b[0], b[1]);
                 }
                 const uint32_t cmb = pack_bf16x2(em[0], em[1]);
 #pragma unroll
@@ -529,26 +559,26 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     uint32_t qw = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_Q + sw128_offset(t, ch0, 8192));
                     uint32_t kw = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_K + sw128_offset(t, ch0, 8192));
                     if (kPacked && t >= nvalid) qw = kw = 0u;
-                    float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xFFFF0000u);
-                    float k0 = __uint_as_float(kw << 16), k1 = __uint_as_float(kw & 0xFFFF0000u);
+                    float2 qv = make_float2(__uint_as_float(qw << 16), __uint_as_float(qw & 0xFFFF0000u));
+                    float2 kv = make_float2(__uint_as_float(kw << 16), __uint_as_float(kw & 0xFFFF0000u));
                     if (kFused) {
                         const float qn = s_norm[t], kn = s_norm[kC + t];
-                        q0 *= qn; q1 *= qn; k0 *= kn; k1 *= kn;
+                        qv = mul2(qv, make_float2(qn, qn));
+                        kv = mul2(kv, make_float2(kn, kn));
                     }
-                    const float x0 = fmaf(gam[i][0], kLog2e, -gmL[0]);
-                    const float x1 = fmaf(gam[i][1], kLog2e, -gmL[1]);
-                    const float E0 = ex2_approx(x0), E1 = ex2_approx(x1);
-                    const float I0 = ex2_approx(-x0), I1 = ex2_approx(-x1);
-                    const float kI0 = k0 * I0, kI1 = k1 * I1;
+                    const float2 x = fma2(gam[i], make_float2(kLog2e, kLog2e), ngmL);
+                    const float2 E = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    const float2 I = make_float2(ex2_approx(-x.x), ex2_approx(-x.y));
+                    const float2 kI = mul2(kv, I);
                     // MMA1 operands: A rows [Qt0;Kt0;Qt1;Kt1], B rows [Kh0(16);Kh1(48);Kh0(48)].  Without
                     // the prologue q and k are bf16 already: bf16 q (k) times the bf16-rounded factor
                     uint32_t a1q, a1k, b1;
                     if (kFused) {
-                        a1q = pack_bf16x2(q0 * E0, q1 * E1);
-                        a1k = pack_bf16x2(k0 * E0, k1 * E1);
-                        b1 = pack_bf16x2(kI0, kI1);
+                        a1q = pack_bf16x2(mul2(qv, E));
+                        a1k = pack_bf16x2(mul2(kv, E));
+                        b1 = pack_bf16x2(kI);
                     } else {
-                        const uint32_t e2 = pack_bf16x2(E0, E1), i2 = pack_bf16x2(I0, I1);
+                        const uint32_t e2 = pack_bf16x2(E), i2 = pack_bf16x2(I);
                         a1q = mul_bf16x2(qw, e2);
                         a1k = mul_bf16x2(kw, e2);
                         b1 = mul_bf16x2(kw, i2);
@@ -561,11 +591,11 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     // so a factor flushes to zero only when the exact product is below the fp32 range
                     if (hq == 0)
                         *reinterpret_cast<uint32_t*>(sm + OFF_BB + sw128_offset(64 + t, ch0, 12288)) =
-                            pack_bf16x2((kI0 * f1[0]) * f2[0], (kI1 * f1[1]) * f2[1]);
+                            pack_bf16x2(mul2(mul2(kI, f1), f2));
                     // MMA3 operand, the same rows against the chunk start: the bf16 tile times bf16 e^{Gam_m}
                     *reinterpret_cast<uint32_t*>(sm + OFF_KQ + sw128_offset(rq, ch0, 16384)) = mul_bf16x2(a1q, cmb);
                     *reinterpret_cast<uint32_t*>(sm + OFF_KQ + sw128_offset(rk, ch0, 16384)) = mul_bf16x2(a1k, cmb);
-                    kb[i] = pack_bf16x2(kI0 * ce[0], kI1 * ce[1]);
+                    kb[i] = pack_bf16x2(mul2(kI, ce));
                 }
             }
             fence_proxy_async_smem();
@@ -630,7 +660,11 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     const float br = s_beta[r];
                     float w[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) w[j] = (jb + j < r) ? br * row[j] : 0.f;
+                    for (int j = 0; j < 32; j += 2) {
+                        const float2 pr = mul2(make_float2(row[j], row[j + 1]), make_float2(br, br));
+                        w[j] = (jb + j < r) ? pr.x : 0.f;
+                        w[j + 1] = (jb + j + 1 < r) ? pr.y : 0.f;
+                    }
 #pragma unroll
                     for (int j = 0; j < 32; j += 8)
                         *reinterpret_cast<uint4*>(sm + OFF_AOFF + r * kLdA * 2 + (jb + j) * 2) = pack8(w + j);
@@ -688,7 +722,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         const float x0 = xm[nt][2 * hr], x1 = xm[nt][2 * hr + 1];
                         *reinterpret_cast<uint32_t*>(sm + OFF_XD + ((o0 + row) * kLdX + col) * 2) = pack_bf16x2(x0, x1);
                         *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(o0 + row), o0 + col, 8192)) =
-                            pack_bf16x2(x0 * b0, x1 * b1);
+                            pack_bf16x2(mul2(make_float2(x0, x1), make_float2(b0, b1)));
                     }
                 }
             }
@@ -784,9 +818,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     float y[8];
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
-                        const float2 f = __bfloat1622float2(v2[m]);
-                        y[2 * m] = f.x - ks[j + 2 * m];
-                        y[2 * m + 1] = f.y - ks[j + 2 * m + 1];
+                        const float2 yy = sub2(__bfloat1622float2(v2[m]), make_float2(ks[j + 2 * m], ks[j + 2 * m + 1]));
+                        y[2 * m] = yy.x;
+                        y[2 * m + 1] = yy.y;
                     }
                     *reinterpret_cast<uint4*>(sm + OFF_V + off) = pack8(y);
                 }
@@ -811,7 +845,11 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 tmem_ld64(tlane + TM_S + 64 * colhalf, sv);
                 const float gc = s_gamma[par][32 * quarter + lane];
 #pragma unroll
-                for (int j = 0; j < 64; ++j) sv[j] *= gc;
+                for (int j = 0; j < 64; j += 2) {
+                    const float2 d = mul2(make_float2(sv[j], sv[j + 1]), make_float2(gc, gc));
+                    sv[j] = d.x;
+                    sv[j + 1] = d.y;
+                }
 #pragma unroll
                 for (int cb = 0; cb < 64; cb += 16) tmem_st16(tlane + TM_S + 64 * colhalf + cb, sv + cb);
                 tmem_wait_st();
