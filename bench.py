@@ -210,23 +210,29 @@ def weak_scaling_throughput(units_per_rank, world, steps, seconds):
 
 
 def measure_e2e(kda, dist, world, dev, stream, args, q, k, v, g, beta, S0, o):
-    """Prefill through the public API with pinned host inputs copied in and o copied out, per step."""
+    """Prefill through the host-buffer entry point, per step: pinned host inputs and S0 copied in,
+    o copied out (the library overlaps copy-in, kernels and copy-out segment by segment)."""
     import torch
     P = PREFILL
     host_in = [t.to("cpu").pin_memory() for t in (q, k, v, g, beta)]
     host_s0 = S0.to("cpu").pin_memory()
     host_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    ws = torch.empty(kda.host_workspace_bytes(P["T"], P["H"], P["dk"], P["dv"], q.dtype), dtype=torch.uint8,
+                     device=dev)
     e2e_steps = max(1, min(args.steps, 3))
+
+    def step():
+        kda.kda_forward_chunked_host(*host_in, host_s0, o=host_o, return_state=False, workspace=ws, stream=stream)
+
+    step()   # untimed: first touch of the workspace
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        dq, dk_, dv_, dg, db = (t.to(dev, non_blocking=True) for t in host_in)
-        ds0 = host_s0.to(dev, non_blocking=True)
-        oo, _ = kda.kda_forward_chunked(dq, dk_, dv_, dg, db, ds0, stream=stream)
-        host_o.copy_(oo, non_blocking=True)
+        step()
     e1.record(stream)
     torch.cuda.synchronize()
     (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], dev, world)
@@ -234,7 +240,8 @@ def measure_e2e(kda, dist, world, dev, stream, args, q, k, v, g, beta, S0, o):
     d2h = host_o.numel() * host_o.element_size()
     return {"value": weak_scaling_throughput(P["B"] * P["T"], world, 1, e2e_ms / 1e3), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "note": "prefill through kda_forward_chunked with pinned host inputs copied in and o copied out"}
+            "note": "prefill through kda_forward_chunked_host: pinned host inputs and S0 in, o out, "
+                    "copies overlapped with the kernels in 2048-token segments"}
 
 
 def run_ours(args):

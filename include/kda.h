@@ -40,6 +40,8 @@
 #ifndef KDA_H_
 #define KDA_H_
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -125,6 +127,46 @@ KDA_API int kda_forward_chunked_states(const void* q, const void* k, const void*
                                const void* beta, const float* S0, void* o, float* S_T,
                                float* S_mid, int interval, int B, int T, int H, int dk, int dv,
                                int dtype, int impl, struct CUstream_st* stream);
+
+/*
+ * kda_forward_chunked_host -- kda_forward_chunked on HOST buffers: the library copies the
+ * inputs in, runs the prefill and copies o (and S_T) out.  The work is cut into segments of
+ * one batch entry and at most 2048 tokens (a multiple of the 64-token chunk); the state passes
+ * from one segment of a sequence to the next in device memory, so o and S_T are bitwise those
+ * of kda_forward_chunked on the same values.  Copy-in of the next segment, the kernel of the
+ * current one and copy-out of the previous one overlap (two internal streams, created and
+ * destroyed by the call, ordered by events with `stream`).
+ *
+ *   q, k, v, g, beta, S0, o, S_T : layouts, dtypes and NULL rules of kda_forward_chunked, in
+ *              HOST memory owned by the caller.  Page-locked memory makes the copies
+ *              asynchronous; with pageable memory they are staged and the call blocks the host
+ *              thread.  S_T may be S0 itself; no other output may overlap an input.  Inputs
+ *              must stay unchanged, and outputs unread, until the work on `stream` completes.
+ *   workspace       : DEVICE memory owned by the caller, 16-byte aligned, of at least
+ *                     kda_forward_chunked_host_workspace(T, H, dk, dv, dtype) bytes; it must
+ *                     not be used by anything else until the work on `stream` completes.
+ *   workspace_bytes : its size.
+ *   impl            : kda_impl, as for kda_forward_chunked_impl.
+ *
+ * Asynchronous on `stream`: everything the call enqueues comes after the work already on
+ * `stream`, and work enqueued on `stream` afterwards comes after all of it (after the last
+ * copy-out).  Returns KDA_OK; KDA_ERR_INVALID_ARG for a missing or too small workspace or a
+ * bad size or overlap; KDA_ERR_MISALIGNED for an unaligned workspace; KDA_ERR_UNSUPPORTED as
+ * kda_forward_chunked_impl (these checks happen before anything is enqueued); KDA_ERR_CUDA if
+ * a stream, event, copy or launch fails part-way (work already enqueued still completes, and
+ * `stream` still waits for it).
+ */
+KDA_API int kda_forward_chunked_host(const void* q, const void* k, const void* v, const void* g,
+                             const void* beta, const float* S0, void* o, float* S_T, int B,
+                             int T, int H, int dk, int dv, int dtype, void* workspace,
+                             size_t workspace_bytes, int impl, struct CUstream_st* stream);
+
+/*
+ * kda_forward_chunked_host_workspace -- bytes of device workspace kda_forward_chunked_host
+ * needs for sequences of T tokens with H heads (independent of B): two segments' inputs and
+ * outputs plus two states.  Returns 0 for an unsupported dtype or head size, H <= 0 or T < 0.
+ */
+KDA_API size_t kda_forward_chunked_host_workspace(int T, int H, int dk, int dv, int dtype);
 
 /*
  * kda_decode_step -- one token for every (b, h), state updated in place.

@@ -7,6 +7,7 @@ these functions raise.
     from linear_attention_recurrence_forward_b200 import kda_forward_chunked, kda_decode_step
     o, S_T = kda_forward_chunked(q, k, v, g, beta, S0)        # prefill, torch CUDA tensors
     o, S_T, S_mid = kda_forward_chunked_states(q, k, v, g, beta, S0, interval=512)
+    o, S_T = kda_forward_chunked_host(q_cpu, k_cpu, v_cpu, g_cpu, beta_cpu, S0_cpu)  # host tensors in and out
     o = kda_decode_step(q, k, v, g, beta, S)                   # one token, S updated in place
 
 Layouts (contiguous): q, k, g [B, T, H, dk]; v, o [B, T, H, dv]; beta [B, T, H];
@@ -24,6 +25,8 @@ import torch
 __all__ = [
     "kda_forward_chunked",
     "kda_forward_chunked_states",
+    "kda_forward_chunked_host",
+    "host_workspace_bytes",
     "kda_decode_step",
     "kda_forward_varlen",
     "kda_forward_chunked_fused",
@@ -78,6 +81,10 @@ def lib() -> ctypes.CDLL:
         L.kda_forward_chunked_impl.restype = I
         L.kda_forward_chunked_states.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]
         L.kda_forward_chunked_states.restype = I
+        L.kda_forward_chunked_host.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, ctypes.c_size_t, I, P]
+        L.kda_forward_chunked_host.restype = I
+        L.kda_forward_chunked_host_workspace.argtypes = [I, I, I, I, I]
+        L.kda_forward_chunked_host_workspace.restype = ctypes.c_size_t
         L.kda_state_compose.argtypes = [P, P, P, P, I, I, I, P]
         L.kda_state_compose.restype = I
         L.kda_forward_chunked_fused.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P]
@@ -157,6 +164,66 @@ def kda_forward_chunked(q, k, v, g, beta, S0=None, *, o=None, S_T=None, return_s
                                             _stream_handle(stream))
     if rc != 0:
         raise KdaError("kda_forward_chunked", rc)
+    return o, S_T
+
+
+def host_workspace_bytes(T: int, H: int, dk: int = 128, dv: int = 128, dtype=torch.bfloat16) -> int:
+    """Bytes of device workspace kda_forward_chunked_host needs for T tokens and H heads."""
+    if dtype not in DTYPE:
+        raise ValueError(f"unsupported dtype {dtype}")
+    n = lib().kda_forward_chunked_host_workspace(int(T), int(H), int(dk), int(dv), DTYPE[dtype])
+    if n == 0:
+        raise ValueError(f"unsupported sizes T={T} H={H} dk={dk} dv={dv}")
+    return int(n)
+
+
+def kda_forward_chunked_host(q, k, v, g, beta, S0=None, *, o=None, S_T=None, return_state: bool = True,
+                             workspace=None, impl: str = "auto", stream=None, device=None):
+    """Prefill over [B, T, H, *] HOST (CPU) tensors, outputs in host memory.
+
+    The library copies the inputs to the GPU segment by segment, runs the prefill and copies o
+    and S_T back, overlapping the copies with the kernels; o and S_T equal kda_forward_chunked's
+    bitwise.  Pinned inputs make the copies asynchronous; outputs allocated here are pinned.
+    The call is asynchronous on `stream`: read o and S_T after synchronizing it.  `workspace` is
+    a CUDA uint8 tensor of at least host_workspace_bytes(T, H, dk, dv, dtype) bytes (allocated on
+    `device` if not given).
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in DTYPE:
+        raise ValueError(f"unsupported dtype {dt}")
+    cpu = torch.device("cpu")
+    for name, t, shape in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("v", v, (B, T, H, dv)),
+                           ("g", g, (B, T, H, dk)), ("beta", beta, (B, T, H))):
+        _check(t, name, shape, dt, cpu)
+    if S0 is not None:
+        _check(S0, "S0", (B, H, dk, dv), torch.float32, cpu)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, pin_memory=True)
+    else:
+        _check(o, "o", (B, T, H, dv), dt, cpu)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, pin_memory=True)
+    elif S_T is not None:
+        _check(S_T, "S_T", (B, H, dk, dv), torch.float32, cpu)
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    nbytes = host_workspace_bytes(T, H, dk, dv, dt)
+    own_workspace = workspace is None
+    if own_workspace:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    elif not (isinstance(workspace, torch.Tensor) and workspace.is_cuda and workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    with torch.cuda.device(workspace.device):
+        rc = lib().kda_forward_chunked_host(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                                            _ptr(S_T), B, T, H, dk, dv, DTYPE[dt], _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(), IMPL[impl],
+                                            _stream_handle(stream))
+        if rc != 0:
+            raise KdaError("kda_forward_chunked_host", rc)
+        if own_workspace and stream is not None:
+            workspace.record_stream(stream)   # not reused before the call's work on `stream` is done
     return o, S_T
 
 

@@ -157,6 +157,161 @@ int forward_impl(const void* q, const void* k, const void* v, const void* g, con
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ host-buffer prefill
+//
+// The work is cut into segments of one batch entry and at most kHostSegTokens tokens (a
+// multiple of the 64-token chunk, so the chunking is that of the whole sequence).  Segment i
+// uses activation slot i % 2 of the workspace and batch entry b the state slot b % 2, which
+// carries the fp32 state from one segment of b to the next (the kernel updates it in place).
+// Three streams overlap the copy-in of segment i+1 and the copy-out of segment i-1 with the
+// kernel of segment i: inputs go in on one internal stream, the kernels run on the caller's
+// stream, outputs come out on a second internal stream, ordered by events.
+constexpr int kHostSegTokens = 2048;
+
+size_t round_up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct HostPlan {
+    int L;                                  // tokens per segment (the last one of a sequence may be shorter)
+    size_t q, v, beta;                      // bytes of a slot's q (= k = g), v (= o) and beta buffers
+    size_t slot, state, total;
+};
+
+HostPlan host_plan(int T, int H, int dk, int dv, int dtype) {
+    HostPlan p{};
+    const size_t es = elem_size(dtype);
+    p.L = T < kHostSegTokens ? T : kHostSegTokens;
+    const size_t n = (size_t)p.L * H;
+    p.q = round_up256(n * dk * es);
+    p.v = round_up256(n * dv * es);
+    p.beta = round_up256(n * es);
+    p.slot = 3 * p.q + 2 * p.v + p.beta;
+    p.state = round_up256((size_t)H * dk * dv * sizeof(float));
+    p.total = 2 * p.slot + 2 * p.state;
+    return p;
+}
+
+int validate_host(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                  const float* S0, const void* o, const float* ST, int B, int T, int H, int dk, int dv,
+                  int dtype, const void* ws, size_t ws_bytes, int impl) {
+    if (impl != KDA_IMPL_AUTO && impl != KDA_IMPL_TCGEN05 && impl != KDA_IMPL_SIMT) return KDA_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || T < 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_FP32) return KDA_ERR_UNSUPPORTED;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    const double elems = (double)B * (double)T * (double)H * (double)(dk > dv ? dk : dv);
+    if (elems > 9.0e15) return KDA_ERR_INVALID_ARG;
+    if (!ws) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(ws)) return KDA_ERR_MISALIGNED;
+    if (ws_bytes < host_plan(T, H, dk, dv, dtype).total) return KDA_ERR_INVALID_ARG;
+    // the host buffers: outputs overlap no input (S_T may be S0 itself)
+    const size_t es = elem_size(dtype);
+    const size_t n_tok = (size_t)B * T * H;
+    const size_t sbytes = (size_t)B * H * dk * dv * sizeof(float);
+    const Range ins[] = {range_of(q, T ? n_tok * dk * es : 0), range_of(k, T ? n_tok * dk * es : 0),
+                         range_of(v, T ? n_tok * dv * es : 0), range_of(g, T ? n_tok * dk * es : 0),
+                         range_of(beta, T ? n_tok * es : 0)};
+    const Range ro = range_of(o, T ? n_tok * dv * es : 0);
+    for (const Range& r : ins)
+        if (overlaps(ro, r)) return KDA_ERR_INVALID_ARG;
+    if (S0 && overlaps(ro, range_of(S0, sbytes))) return KDA_ERR_INVALID_ARG;
+    if (ST) {
+        const Range rs = range_of(ST, sbytes);
+        if (overlaps(rs, ro)) return KDA_ERR_INVALID_ARG;
+        for (const Range& r : ins)
+            if (overlaps(rs, r)) return KDA_ERR_INVALID_ARG;
+        if (S0 && S0 != ST && overlaps(rs, range_of(S0, sbytes))) return KDA_ERR_INVALID_ARG;
+    }
+    return KDA_OK;
+}
+
+int forward_host_impl(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                      const float* S0, void* o, float* ST, int B, int T, int H, int dk, int dv, int dtype,
+                      void* ws, size_t ws_bytes, int impl, cudaStream_t stream) {
+    int rc = validate_host(q, k, v, g, beta, S0, o, ST, B, T, H, dk, dv, dtype, ws, ws_bytes, impl);
+    if (rc != KDA_OK) return rc;
+    const HostPlan P = host_plan(T, H, dk, dv, dtype);
+    const size_t es = elem_size(dtype);
+    const size_t sbytes = (size_t)H * dk * dv * sizeof(float);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    float* state[2] = {reinterpret_cast<float*>(base + 2 * P.slot),
+                       reinterpret_cast<float*>(base + 2 * P.slot + P.state)};
+    if (T == 0) {
+        // no tokens: S_T = S0 (or zeros), through a state slot, in order on the caller's stream
+        if (!ST) return KDA_OK;
+        for (int b = 0; b < B; ++b) {
+            cudaError_t e = S0 ? cudaMemcpyAsync(state[0], S0 + (size_t)b * H * dk * dv, sbytes,
+                                                 cudaMemcpyHostToDevice, stream)
+                               : cudaMemsetAsync(state[0], 0, sbytes, stream);
+            if (e == cudaSuccess)
+                e = cudaMemcpyAsync(ST + (size_t)b * H * dk * dv, state[0], sbytes, cudaMemcpyDeviceToHost, stream);
+            if (e != cudaSuccess) return KDA_ERR_CUDA;
+        }
+        return KDA_OK;
+    }
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev[8] = {};   // start, in[2], done[2], out[2], end
+    bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess;
+    for (int i = 0; i < 8 && ok; ++i) ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+    cudaEvent_t ev_start = ev[0], ev_end = ev[7];
+    cudaEvent_t ev_in[2] = {ev[1], ev[2]}, ev_done[2] = {ev[3], ev[4]}, ev_out[2] = {ev[5], ev[6]};
+    // everything this call enqueues follows the work already on the caller's stream
+    if (ok) ok = cudaEventRecord(ev_start, stream) == cudaSuccess &&
+                 cudaStreamWaitEvent(s_in, ev_start, 0) == cudaSuccess;
+    auto h2d = [&](void* dst, const void* src, size_t n) {
+        if (ok) ok = cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, s_in) == cudaSuccess;
+    };
+    auto d2h = [&](void* dst, const void* src, size_t n) {
+        if (ok) ok = cudaMemcpyAsync(dst, src, n, cudaMemcpyDeviceToHost, s_out) == cudaSuccess;
+    };
+    bool out_pending[2] = {false, false};
+    int seg = 0;
+    for (int b = 0; b < B && ok && rc == KDA_OK; ++b) {
+        float* Sb = state[b & 1];
+        for (int t0 = 0; t0 < T && ok && rc == KDA_OK; t0 += P.L, ++seg) {
+            const int L = T - t0 < P.L ? T - t0 : P.L;
+            const int s = seg & 1;
+            uint8_t* sl = base + (size_t)s * P.slot;
+            uint8_t *dq = sl, *dk_ = sl + P.q, *dg = sl + 2 * P.q, *dv_ = sl + 3 * P.q;
+            uint8_t *dbeta = dv_ + P.v, *do_ = dbeta + P.beta;
+            const size_t th = ((size_t)b * T + t0) * H;   // first token-head of the segment
+            const size_t n = (size_t)L * H;
+            // copy-in: the slot (and the state slot of batch entry b - 2) is free once the segment
+            // two back has been copied out
+            if (out_pending[s] && ok) ok = cudaStreamWaitEvent(s_in, ev_out[s], 0) == cudaSuccess;
+            h2d(dq, static_cast<const uint8_t*>(q) + th * dk * es, n * dk * es);
+            h2d(dk_, static_cast<const uint8_t*>(k) + th * dk * es, n * dk * es);
+            h2d(dg, static_cast<const uint8_t*>(g) + th * dk * es, n * dk * es);
+            h2d(dv_, static_cast<const uint8_t*>(v) + th * dv * es, n * dv * es);
+            h2d(dbeta, static_cast<const uint8_t*>(beta) + th * es, n * es);
+            if (t0 == 0 && S0) h2d(Sb, S0 + (size_t)b * H * dk * dv, sbytes);
+            if (ok) ok = cudaEventRecord(ev_in[s], s_in) == cudaSuccess &&
+                         cudaStreamWaitEvent(stream, ev_in[s], 0) == cudaSuccess;
+            if (!ok) break;
+            // the prefill of the segment, from the carried state (or S0 / zeros at the start)
+            const float* s_from = (t0 == 0 && !S0) ? nullptr : Sb;
+            rc = forward_impl(dq, dk_, dv_, dg, dbeta, s_from, do_, Sb, 1, L, H, dk, dv, dtype, impl, stream);
+            if (rc != KDA_OK) break;
+            ok = cudaEventRecord(ev_done[s], stream) == cudaSuccess &&
+                 cudaStreamWaitEvent(s_out, ev_done[s], 0) == cudaSuccess;
+            // copy-out of o, and of the final state after the last segment of b
+            d2h(static_cast<uint8_t*>(o) + th * dv * es, do_, n * dv * es);
+            if (ST && t0 + L == T) d2h(ST + (size_t)b * H * dk * dv, Sb, sbytes);
+            if (ok) ok = cudaEventRecord(ev_out[s], s_out) == cudaSuccess;
+            out_pending[s] = true;
+        }
+    }
+    // the caller's stream continues only after every copy-out (also after a failure part-way)
+    if (ev_end && s_out && cudaEventRecord(ev_end, s_out) == cudaSuccess)
+        (void)cudaStreamWaitEvent(stream, ev_end, 0);
+    for (cudaEvent_t e : ev)
+        if (e) cudaEventDestroy(e);   // released once complete
+    if (s_in) cudaStreamDestroy(s_in);
+    if (s_out) cudaStreamDestroy(s_out);
+    if (rc != KDA_OK) return rc;
+    return ok ? KDA_OK : KDA_ERR_CUDA;
+}
+
 int decode_impl(const void* q, const void* k, const void* v, const void* g, const void* beta, float* S,
                 int n_slots, const int* slots, void* o, int B, int H, int dk, int dv, int dtype,
                 cudaStream_t stream) {
@@ -227,6 +382,20 @@ int kda_forward_varlen(const void* q, const void* k, const void* v, const void* 
     if (N <= 0 || !cu_seqlens) return KDA_ERR_INVALID_ARG;
     return forward_impl(q, k, v, g, beta, S0, o, S_T, N, T_total, H, dk, dv, dtype, impl, stream, nullptr, 0,
                         cu_seqlens);
+}
+
+size_t kda_forward_chunked_host_workspace(int T, int H, int dk, int dv, int dtype) {
+    if (T < 0 || H <= 0 || !head_dim_ok(dk) || !head_dim_ok(dv) ||
+        (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_FP32))
+        return 0;
+    return host_plan(T, H, dk, dv, dtype).total;
+}
+
+int kda_forward_chunked_host(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                             const float* S0, void* o, float* S_T, int B, int T, int H, int dk, int dv,
+                             int dtype, void* workspace, size_t workspace_bytes, int impl, cudaStream_t stream) {
+    return forward_host_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, dtype, workspace, workspace_bytes,
+                             impl, stream);
 }
 
 int kda_decode_step(const void* q, const void* k, const void* v, const void* g, const void* beta,
