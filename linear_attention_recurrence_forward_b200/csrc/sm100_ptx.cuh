@@ -51,10 +51,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 }
 
 // Wait for the phase with the given parity to complete; give up after `timeout_ns`
-// of wall time (returns false).  Never traps, never spins forever.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
-    const uint32_t a = smem_u32(bar);
-    if (mbar_try_wait(a, parity)) return true;
+// of wall time (returns false).  Never traps, never spins forever.  The first test is inline;
+// the timed retry loop is one out-of-line copy, which keeps the callers' loops (and their
+// instruction-cache footprint) smaller.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t a, uint32_t parity, uint64_t timeout_ns) {
     const uint64_t t0 = global_timer_ns();
     for (;;) {
 #pragma unroll 1
@@ -62,6 +62,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
             if (mbar_try_wait(a, parity)) return true;
         if (global_timer_ns() - t0 > timeout_ns) return false;
     }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    return mbar_wait_slow(a, parity, timeout_ns);
 }
 
 // ------------------------------------------------------------------ named barriers
