@@ -138,6 +138,18 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sms)}
 
 
+def cpu_model():
+    """The host CPU's model name (Linux), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def oracle_baseline(budget_s=15.0, seed=0):
     """Time the fp64 oracle (as it stands) on a bounded sample of the prefill workload.
 
@@ -163,9 +175,19 @@ def oracle_baseline(budget_s=15.0, seed=0):
     oracle.forward(q, k, v, g, beta, S0, nthreads=cores)
     dt = time.perf_counter() - t0
     token_heads_per_s = n_heads * T / dt
+    # one thread on one head of the 4096-token, 32-head workload
+    T1, H1 = 4096, 32
+    one = make_prefill_inputs(1, T1, 1, d, d, "bf16", seed=seed + 2)
+    t1 = time.perf_counter()
+    oracle.forward(*one[:5], None, nthreads=1)
+    dt1 = time.perf_counter() - t1
     return {"value": token_heads_per_s / H, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"{n_heads} heads x {T} tokens of the K3 prefill workload (d=128), fp64, {dt:.1f} s; "
                       f"tokens/s = token-heads/s / {H}",
+            "cpu_model": cpu_model(),
+            "single_thread": {"value": T1 / dt1 / H1, "unit": "tokens/s", "threads": 1,
+                              "sample": f"1 head x {T1} tokens of the h32_t4k workload (B1 T4096 H32 d128), "
+                                        f"fp64, {dt1:.2f} s; tokens/s = token-heads/s / {H1}"},
             "seconds": dt, "token_heads_per_s": token_heads_per_s}
 
 
@@ -188,7 +210,8 @@ def run_reference(args):
             "config": {"workload": PREFILL["name"], "B": PREFILL["B"], "T": PREFILL["T"], "H": PREFILL["H"],
                        "dk": PREFILL["dk"], "dv": PREFILL["dv"]},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": base["cores"], "kind": "oracle",
-                             "sample": base["sample"]},
+                             "sample": base["sample"], "cpu_model": base["cpu_model"],
+                             "single_thread": base["single_thread"]},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -400,7 +423,7 @@ def run_ours(args):
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = oracle_baseline(budget_s=args.cpu_budget)
-        cpu = {k_: cpu[k_] for k_ in ("value", "unit", "cores", "kind", "sample")}
+        cpu = {k_: cpu[k_] for k_ in ("value", "unit", "cores", "kind", "sample", "cpu_model", "single_thread")}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
