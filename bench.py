@@ -47,6 +47,23 @@ def decode_alg_bytes(batch, H, dk, dv, elem=2):
     return batch * H * (2 * 4 * dk * dv + elem * (3 * dk + dv) + elem + elem * dv)
 
 
+# Contraction work of the chunked prefill per token-head (d = 128, chunk 64): the three state
+# products at 2 d^2 each, plus five 64 x 64 x d products counted causally (half) or as whole tiles.
+PREFILL_FLOP_CAUSAL = 6 * 128 * 128 + 5 * 64 * 128
+PREFILL_FLOP_DENSE = 6 * 128 * 128 + 10 * 64 * 128
+
+
+def measured_bf16_tflops():
+    """Measured dense bf16 tensor throughput (burst), or the fallback figure."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -424,6 +441,15 @@ def run_ours(args):
     if world == 1 and not args.no_cpu_baseline:
         cpu = oracle_baseline(budget_s=args.cpu_budget)
         cpu = {k_: cpu[k_] for k_ in ("value", "unit", "cores", "kind", "sample", "cpu_model", "single_thread")}
+    tc_peak, tc_kind = measured_bf16_tflops()
+    token_heads = P["B"] * P["T"] * P["H"]
+    tensor_line = {"unit": "TFLOP/s", "peak": tc_peak, "peak_kind": tc_kind,
+                   "causal": token_heads * PREFILL_FLOP_CAUSAL / (prefill_launch_ms * 1e-3) / 1e12,
+                   "dense_tiles": token_heads * PREFILL_FLOP_DENSE / (prefill_launch_ms * 1e-3) / 1e12,
+                   "note": "contraction work per launch / launch time (139,264 flop per token-head causal, "
+                           "180,224 as whole tiles); the kernel is HBM-bound, so this is context"}
+    tensor_line["frac_causal"] = tensor_line["causal"] / tc_peak
+    tensor_line["frac_dense_tiles"] = tensor_line["dense_tiles"] / tc_peak
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -435,7 +461,7 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": recorded_traffic(impl_tag),
                      "kernel": impl_tag, "alg_bytes_per_launch": pb, "launch_ms": prefill_launch_ms,
-                     "peak_kind": peak_kind},
+                     "peak_kind": peak_kind, "tensor": tensor_line},
         "decode": {"states_per_s": decode_states_per_s, "tokens_per_s": decode_states_per_s / D["H"],
                    "ms_per_step": decode_launch_ms,
                    "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peak, "unit": "GB/s",
