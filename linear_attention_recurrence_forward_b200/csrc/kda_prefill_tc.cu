@@ -790,15 +790,15 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         fence_proxy_async_smem();
         tc_fence_before_sync();
         named_bar_sync(kBarSerial, kSerialThreads);
+        // ---- S1 of chunk 0: MMA3 once the prep group has the operand tiles (later chunks issue it
+        // at the end of the previous chunk)
+        if (stid == 0 && nchunks > 0) {
+            ok = mbar_wait(&bar_kq, 0u, p.timeout_ns);
+            if (ok) issue_for_chunk(0);
+        }
         for (int chunk = 0; chunk < nchunks; ++chunk) {
             const uint32_t par = chunk & 1;
             const int t0 = chunk * kC;
-            // ---- S1: MMA1 and MMA3 once the prep group has the operand tiles (chunk 0 here; later
-            // chunks issue them at the end of the previous chunk)
-            if (stid == 0 && chunk == 0) {
-                ok = mbar_wait(&bar_kq, par, p.timeout_ns);
-                if (ok) issue_for_chunk(0);
-            }
             // Y = V - Kt S (Kt rows sit in lanes 32-63 and 96-127), in place over v
             if (ok) ok = mbar_wait(&bar_c, par, p.timeout_ns);
             if (ok) ok = mbar_wait(&bar_v, par, p.timeout_ns);
