@@ -21,9 +21,10 @@
  *     gated delta rule (Gated DeltaNet), which this library's prefill follows.
  *
  * Conventions shared by every entry point
- *   - All tensor pointers are DEVICE pointers owned by the caller.  The library never
- *     allocates, frees or retains caller memory.  It owns one small static device status
- *     word per device (see kda_get_device_status).
+ *   - All tensor pointers are DEVICE pointers owned by the caller (except in
+ *     kda_forward_chunked_host, which takes HOST buffers and a caller-owned device
+ *     workspace).  The library never allocates, frees or retains caller memory.  It owns one
+ *     small static device status word per device (see kda_get_device_status).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
  *     stream).  A return of KDA_OK means the work was validated and enqueued.
  *   - Tensors are contiguous, row-major, with the layouts stated per function.

@@ -1,4 +1,5 @@
-// C ABI of the KDA library: argument validation, kernel choice, the device status word.
+// C ABI of the KDA library: argument validation, kernel choice, the device status word, and
+// the host-buffer prefill (copy-in, kernels and copy-out pipelined over segments).
 //
 // Everything here runs on the host before a launch; nothing is enqueued unless every
 // check passes.  The kernels themselves live in kda_decode.cu, kda_prefill_simt.cu and

@@ -27,10 +27,12 @@
 // CTA organisation: one (b, h) per CTA, 16 warps, two warp-specialised groups coupled by
 // mbarriers so that the state-independent work of chunk c+1 overlaps the recurrence of
 // chunk c:
-//   prep warps 0..7    per chunk: TMA q,k,g -> Gam = L g (tensor core) -> per-channel
-//                      constants -> bf16 operand tiles -> MMA1 (A and P in one product) ->
-//                      fp32 triangular solve (diagonal blocks by substitution, off-diagonal
-//                      blocks on warp-level bf16 MMA tiles) -> T, P, Kb tiles.
+//   prep warps 0..7    per chunk: Gam as an fp32 running sum in registers (the next chunk's g
+//                      is loaded as soon as it has been read) -> per-channel constants ->
+//                      bf16 operand tiles -> MMA1 (A and P in one product) -> the triangular
+//                      solve on warp-level bf16 MMA tiles (diagonal blocks by a doubling
+//                      product, off-diagonal blocks by a walk down each block column) ->
+//                      T, P, Kb tiles.
 //   serial warps 8..15 per chunk: MMA3 [Qt;Kt] S -> Y = V - Kt S -> MMA4 U = T Y ->
 //                      MMA5 O = Qt S + P U, MMA6 S += Kb^T U (state decayed in TMEM first)
 //                      -> O to global, S to bf16 for the next chunk.
@@ -53,7 +55,7 @@ constexpr int kThreads = 512;   // 16 warps
 constexpr int kPrepThreads = 256;
 constexpr int kSerialThreads = 256;
 constexpr uint32_t kBarPrep = 1, kBarSerial = 2;   // named hardware barriers
-constexpr int kIssuer = 0;                         // prep thread that issues the first TMA load and signals
+constexpr int kIssuer = 0;                         // prep thread that issues the g loads (and chunk 0's q, k) and signals
 constexpr int kMma1Issuer = 224;                   // prep thread that issues MMA1 (warp 7: lightest in the solve)
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
@@ -426,7 +428,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         unsigned short beta_next = fetch_beta(0);
         for (int chunk = 0; chunk < nchunks; ++chunk) {
             const uint32_t par = chunk & 1, ppar = par ^ 1u;
-            // ---- P1: beta; this chunk's q, k, g
+            // ---- P1: beta; this chunk's g
             if (ptid < kC) {
                 const float bz = __uint_as_float((uint32_t)beta_next << 16);
                 // with the prologue beta is a logit; a padding token keeps beta = 0
@@ -608,8 +610,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 issue_mma<8, false, 16384, false, 12288>(tbase + TM_P, sb + OFF_A1, sb + OFF_BB, ID_MMA1, false);
                 mma_commit(&bar_ap);
             }
-            // KQ of this chunk is ready and its raw q, k, g consumed: the recurrence group's leader
-            // issues MMA3 and the next chunk's loads
+            // KQ of this chunk is ready and its raw q, k consumed: the recurrence group's leader
+            // issues MMA3 and the next chunk's q, k loads
             if (ptid == kIssuer && !(p.skip_handoff && chunk == 0)) mbar_arrive(&bar_kq);
             // ---- P4: Kb tile, P and A from TMEM, triangular solve, T tile
             if (chunk > 0) ok = mbar_wait(&bar_os, ppar, p.timeout_ns);  // T, P, Kb released
@@ -756,7 +758,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         int pending = -1;                                   // chunk whose v load is in flight
         int pending_qk = -1;                                // last chunk whose q,k loads this leader issued
         // Once the prep group has published chunk c's operand tiles (bar_kq): MMA3 = [Qt0;Kt0;Qt1;Kt1] S
-        // and the raw q, k, g of chunk c+1 into the buffers the prep group has finished reading.
+        // and the raw q, k of chunk c+1 into the buffers the prep group has finished reading.
         auto issue_for_chunk = [&](int c) {
             tc_fence_after_sync();
             issue_mma<8, false, 16384, true, 16384>(tbase + TM_C, sb + OFF_KQ, sb + OFF_SB, ID_KxMN, false);
