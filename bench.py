@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 METRIC = "KDA prefill tokens/s (K3 shape, H=96, d=128) and decode states/s; % of roofline"
 PREFILL = dict(name="k3_b4_t8k", B=4, T=8192, H=96, dk=128, dv=128, dtype="bf16", s0_std=0.02, zg_mean=-2.0)
 DECODE = dict(name="decode_b256_h96", batch=256, H=96, dk=128, dv=128, dtype="bf16")
+LONG = dict(name="k3_t64k", B=1, T=65536, H=96, dk=128, dv=128, dtype="bf16")
 DECODE_RING = 8
 
 
@@ -413,6 +414,38 @@ def run_ours(args):
                               "(an unfused pipeline also reads and writes them once more in a separate pass)"}
         del raw
 
+    # ---- the long-context workload (B1 T65536 H96, S0 = 0, 1024 chunks carried in sequence), timed alone
+    long_line = None
+    if not args.no_long:
+        LC = LONG
+        lq = make_prefill_inputs(LC["B"], LC["T"], LC["H"], LC["dk"], LC["dv"], LC["dtype"], seed=4000 + rank,
+                                 device=str(dev))
+        lo = torch.empty((LC["B"], LC["T"], LC["H"], LC["dv"]), dtype=lq[0].dtype, device=dev)
+        lst = torch.empty((LC["B"], LC["H"], LC["dk"], LC["dv"]), dtype=torch.float32, device=dev)
+        for _ in range(2):
+            kda.kda_forward_chunked(*lq[:5], None, o=lo, S_T=lst, stream=stream)
+        reps = max(3, min(args.steps, 10))
+        lev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        torch.cuda.synchronize()
+        for e0, e1 in lev:
+            e0.record(stream)
+            kda.kda_forward_chunked(*lq[:5], None, o=lo, S_T=lst, stream=stream)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        if kda.kda_get_device_status() != 0:
+            raise RuntimeError("device status after the long-context run")
+        l_ms = sum(e0.elapsed_time(e1) for e0, e1 in lev) / reps
+        lb = prefill_alg_bytes(LC["B"], LC["T"], LC["H"], LC["dk"], LC["dv"], with_s0=False)
+        lpeak, lpeak_kind = measured_peaks()
+        l_ach = lb / (l_ms / 1e3) / 1e9
+        long_line = {"workload": LC["name"], "B": LC["B"], "T": LC["T"], "H": LC["H"], "launch_ms": l_ms,
+                     "tokens_per_s": LC["B"] * LC["T"] / (l_ms / 1e3), "launches": reps,
+                     "roofline": {"bound": "hbm", "achieved": l_ach, "peak": lpeak, "unit": "GB/s",
+                                  "frac": l_ach / lpeak, "alg_bytes_per_launch": lb, "peak_kind": lpeak_kind},
+                     "grid": f"{LC['B'] * LC['H']} CTAs (one per head) on the SMs",
+                     "timed": "separately, after the headline region, CUDA events per launch"}
+        del lq, lo, lst
+
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
     if args.no_e2e:
         e2e = None
@@ -467,6 +500,7 @@ def run_ours(args):
                    "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peak, "unit": "GB/s",
                                 "frac": dec_achieved / peak, "alg_bytes_per_launch": db_,
                                 "traffic": recorded_traffic("decode")}},
+        "long_context": long_line,
         "state_emission": states_line,
         "fused_prologue": fused_line,
         "cpu_baseline": cpu,
@@ -493,6 +527,7 @@ def main():
     ap.add_argument("--decode-batch", type=int, default=None, help="override the decode batch (profiling)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-states", action="store_true", help="skip the state-emission (every 512 tokens) timing")
+    ap.add_argument("--no-long", action="store_true", help="skip the long-context (T = 65536) timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -69,9 +69,12 @@ typedef enum { KDA_DTYPE_BF16 = 0, KDA_DTYPE_FP32 = 1 } kda_dtype;
 
 /* Prefill kernel selection for kda_forward_chunked_impl. */
 typedef enum {
-    KDA_IMPL_AUTO = 0,    /* tcgen05 kernel when it supports the shape, else the SIMT kernel */
+    KDA_IMPL_AUTO = 0,    /* bf16 inputs: the tcgen05 kernel (dk = dv = 128; any other bf16 head size
+                             is refused with KDA_ERR_UNSUPPORTED, never run token-serially without
+                             being asked); fp32 inputs: the SIMT kernel (the only fp32 kernel: bf16
+                             tensor-core operands cannot meet an fp32 accuracy bar) */
     KDA_IMPL_TCGEN05 = 1, /* chunkwise tensor-core kernel: bf16, dk = dv = 128 only */
-    KDA_IMPL_SIMT = 2     /* fp32 CUDA-core kernel: every supported dtype and size */
+    KDA_IMPL_SIMT = 2     /* token-serial fp32 CUDA-core kernel: every supported dtype and size */
 } kda_impl;
 
 /*
@@ -89,6 +92,10 @@ typedef enum {
  *             S_T may alias S0 exactly (in-place state carry); any other overlap
  *             between outputs and inputs is not allowed.
  *   dtype   : kda_dtype.
+ *
+ * Kernel: KDA_IMPL_AUTO (see kda_impl): bf16 with dk = dv = 128 runs the chunkwise tensor-core
+ * kernel, fp32 the fp32 kernel; bf16 with another head size returns KDA_ERR_UNSUPPORTED (use
+ * kda_forward_chunked_impl with KDA_IMPL_SIMT for it).
  *
  * Returns KDA_OK, or a negative kda_status (nothing is enqueued on error).
  */
@@ -218,9 +225,11 @@ KDA_API int kda_forward_chunked_fused(const void* q_raw, const void* k_raw, cons
  *   v          : [T_total, H, dv]   dtype
  *   beta       : [T_total, H]       dtype
  *   cu_seqlens : [N + 1] int32 DEVICE array: sequence n is tokens cu_seqlens[n] .. cu_seqlens[n+1]-1,
- *                0 <= cu_seqlens[n] <= cu_seqlens[n+1] <= T_total.  The kernels check it: a sequence
- *                whose range is invalid is processed as empty (S_T = S0) and the device status word
- *                is set to KDA_ERR_INVALID_ARG.  o rows of tokens outside every range are not written.
+ *                with 0 <= cu_seqlens[0] <= cu_seqlens[1] <= ... <= cu_seqlens[N] <= T_total (so no two
+ *                sequences share a token; gaps between them are allowed).  The kernels check the whole
+ *                array: if it breaks any of these rules, EVERY sequence is processed as empty (S_T = S0,
+ *                no o row written) and the device status word is set to KDA_ERR_INVALID_ARG.  o rows of
+ *                tokens outside every range are not written.
  *   S0, S_T    : [N, H, dk, dv] fp32, S0 may be NULL (zeros), S_T may be NULL or alias S0
  *   o          : [T_total, H, dv]   dtype
  *   impl       : kda_impl.
@@ -275,6 +284,13 @@ KDA_API int kda_state_compose(const float* M, const float* S_in, const float* N,
  * outputs are then undefined), KDA_ERR_INVALID_ARG (a kernel found an out-of-range device
  * index: a sequence offset or a state slot), or KDA_ERR_CUDA if the synchronisation itself
  * failed.
+ *
+ * The word belongs to the DEVICE, not to a call or a stream: every kernel of the library on that
+ * device, on any stream, sets the same word (the first error wins), and a read clears it.  Only
+ * `stream` is synchronised, so with work on several streams a kernel still running on another one
+ * may set the word after the read, and the error read may come from another stream's call.  When
+ * several streams are in use, synchronise the device (cudaDeviceSynchronize) before calling this
+ * to attribute an error to the work enqueued before that point.
  */
 KDA_API int kda_get_device_status(struct CUstream_st* stream);
 

@@ -141,6 +141,10 @@ int forward_impl(const void* q, const void* k, const void* v, const void* g, con
                        interval, n_mid, cu_seqlens, fused};
     const bool tc_ok = kda::prefill_tc_supports(a);
     if (impl == KDA_IMPL_TCGEN05 && !tc_ok) return KDA_ERR_UNSUPPORTED;
+    // AUTO: the chunkwise tensor-core kernel for bf16 (dk = dv = 128), the fp32 kernel for fp32
+    // inputs; a bf16 shape the tensor-core kernel does not cover is refused rather than sent to the
+    // token-serial kernel behind the caller's back (KDA_IMPL_SIMT runs it when asked for)
+    if (impl == KDA_IMPL_AUTO && dtype == KDA_DTYPE_BF16 && !tc_ok) return KDA_ERR_UNSUPPORTED;
     if (T == 0) {
         // No tokens: the final state is the initial state.
         if (!ST) return KDA_OK;
@@ -153,7 +157,7 @@ int forward_impl(const void* q, const void* k, const void* v, const void* g, con
     a.status = status_word_for_current_device();
     if (!a.status) return KDA_ERR_CUDA;
     cudaError_t e;
-    if (impl == KDA_IMPL_SIMT || (impl == KDA_IMPL_AUTO && !tc_ok)) e = kda::launch_prefill_simt(a, stream);
+    if (impl == KDA_IMPL_SIMT || (impl == KDA_IMPL_AUTO && dtype == KDA_DTYPE_FP32)) e = kda::launch_prefill_simt(a, stream);
     else e = kda::launch_prefill_tc(a, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

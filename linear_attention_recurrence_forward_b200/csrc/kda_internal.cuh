@@ -72,6 +72,18 @@ __device__ __forceinline__ void store_elem(__nv_bfloat16* p, size_t i, float x) 
     p[i] = __float2bfloat16_rn(x);
 }
 
+// Whether packed-sequence offsets form one valid layout, 0 <= cu[0] <= cu[1] <= ... <= cu[n] <= T
+// (non-decreasing, so no two sequences share a token).  A block-wide vote: every thread of the
+// block must call it, and all of them get the same answer.
+__device__ __forceinline__ bool packed_offsets_valid(const int* cu, int n, int T) {
+    bool ok = true;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int a = cu[i], b = cu[i + 1];
+        ok = ok && a <= b && (i > 0 || a >= 0) && (i < n - 1 || b <= T);
+    }
+    return __syncthreads_and(ok) != 0;
+}
+
 // Set the device status word once (first error wins).
 __device__ __forceinline__ void report_status(int* status, int code) {
     if (status) atomicCAS(status, 0, code);

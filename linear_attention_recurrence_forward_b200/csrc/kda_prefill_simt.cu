@@ -47,11 +47,12 @@ kda_prefill_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, co
     size_t base = (size_t)b * T_all;
     int T = T_all;
     if (cu_seqlens) {
-        const int s0 = cu_seqlens[b], s1 = cu_seqlens[b + 1];
-        const bool valid = 0 <= s0 && s0 <= s1 && s1 <= T_all;
+        // offsets that are not one valid layout (one overlapping or out-of-range sequence is
+        // enough) leave every sequence empty and are reported
+        const bool valid = packed_offsets_valid(cu_seqlens, (int)(gridDim.x / NSLICE / H), T_all);
         if (!valid && threadIdx.x == 0) report_status(status, KDA_ERR_INVALID_ARG);
-        base = valid ? (size_t)s0 : 0;
-        T = valid ? s1 - s0 : 0;
+        base = valid ? (size_t)cu_seqlens[b] : 0;
+        T = valid ? cu_seqlens[b + 1] - cu_seqlens[b] : 0;
     }
 
     float4 s[RPT];

@@ -348,16 +348,15 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const int b = bh / p.H, h = bh % p.H;
     // This CTA's tokens: rows tok0 .. tok0 + T - 1 of batch entry bmap of the tensor maps, i.e.
     // [B, T, H, d] as laid out, or sequence b of packed sequences (maps with one batch entry of
-    // all tokens; offsets from cu_seqlens, checked here: an invalid range is reported and
-    // processed as empty)
+    // all tokens; offsets from cu_seqlens, checked here as a whole: offsets that are not one
+    // valid, non-overlapping layout are reported and every sequence is processed as empty)
     int tok0 = 0, bmap = b, T = p.T;
     if (kPacked) {
-        const int s0 = p.cu_seqlens[b], s1 = p.cu_seqlens[b + 1];
-        const bool valid = 0 <= s0 && s0 <= s1 && s1 <= p.T;
+        const bool valid = packed_offsets_valid(p.cu_seqlens, p.B, p.T);
         if (!valid && tid_is_zero()) report_status(p.status, KDA_ERR_INVALID_ARG);
-        tok0 = valid ? s0 : 0;
+        tok0 = valid ? p.cu_seqlens[b] : 0;
         bmap = 0;
-        T = valid ? s1 - s0 : 0;
+        T = valid ? p.cu_seqlens[b + 1] - tok0 : 0;
     }
     const size_t row0 = (size_t)bmap * p.T + tok0;   // token-axis row of this CTA's first token
     const int nchunks = (T + kC - 1) / kC;

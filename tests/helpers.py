@@ -1,5 +1,10 @@
-"""Shared test helpers: the error metric and small seeded-input builders."""
+"""Shared test helpers: the error metric, the parity error log and small seeded-input builders."""
 import numpy as np
+
+# Every parity comparison that goes through check_parity() is recorded here and printed as a
+# table at the end of the pytest session (tests/conftest.py), so a run's log carries the
+# measured errors next to the pass/fail verdict.
+PARITY_LOG = []
 
 
 def max_rel_err(x, ref) -> float:
@@ -20,6 +25,57 @@ def max_rel_err(x, ref) -> float:
     if scale == 0.0:
         return float(err)
     return float(err / scale)
+
+
+def error_stats(x, ref, head_axes=None, floor_frac=1e-2):
+    """Error figures of one output tensor against its reference.
+
+    rel       max|x - ref| / max|ref| (the pass metric)
+    abs       max|x - ref|
+    elem      max_i |x_i - ref_i| / (|ref_i| + floor), floor = floor_frac * max|ref|: the
+              element-wise relative error, with small reference values measured against the floor
+    head_rel  the pass metric per head (the tensor split along `head_axes`, which are kept),
+              worst head: an error confined to the small-magnitude heads shows here
+    """
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert x.shape == ref.shape, (x.shape, ref.shape)
+    if x.size == 0:
+        return dict(rel=0.0, abs=0.0, elem=0.0, head_rel=0.0)
+    if not np.all(np.isfinite(x)):
+        inf = float("inf")
+        return dict(rel=inf, abs=inf, elem=inf, head_rel=inf)
+    d = np.abs(x - ref)
+    a = np.abs(ref)
+    scale = float(a.max())
+    out = dict(rel=max_rel_err(x, ref), abs=float(d.max()))
+    out["elem"] = float(np.max(d / (a + floor_frac * scale))) if scale > 0 else float(d.max())
+    if head_axes:
+        red = tuple(i for i in range(x.ndim) if i not in head_axes)
+        hd, ha = d.max(axis=red), a.max(axis=red)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            r = np.where(ha > 0, hd / np.where(ha > 0, ha, 1.0), hd)
+        out["head_rel"] = float(r.max())
+    else:
+        out["head_rel"] = out["rel"]
+    return out
+
+
+def check_parity(case: str, tensor: str, x, ref, tol: float, head_axes=None, head_tol=None):
+    """Record the error figures of one output tensor and assert the pass bar max rel <= tol
+    (and, when given, the per-head bar head_tol).  Returns the figures."""
+    s = error_stats(x, ref, head_axes=head_axes)
+    PARITY_LOG.append(dict(case=case, tensor=tensor, tol=tol, **s))
+    assert s["rel"] <= tol, f"{case} {tensor}: max rel err {s['rel']:.3e} > {tol:g}"
+    if head_tol is not None:
+        assert s["head_rel"] <= head_tol, f"{case} {tensor}: worst head {s['head_rel']:.3e} > {head_tol:g}"
+    return s
+
+
+def merge_stats(items):
+    """Worst case of several error_stats() results (e.g. one per step or per slice)."""
+    keys = ("rel", "abs", "elem", "head_rel")
+    return {k: max(s[k] for s in items) for k in keys}
 
 
 def unit_rows(rng, shape):

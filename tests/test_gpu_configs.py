@@ -1,8 +1,12 @@
 """The tensor-core prefill and the decode kernel on the five measured workloads (GPU).
 
-Small cases compare every element with the oracle; at full size the comparison runs on
-sampled heads the oracle can afford (whole sequences for those heads), as configured for
-the benchmark launch.  Tolerance: max |x - ref| / max |ref| <= 2e-2 (bf16), 1e-4 (fp32).
+Every workload is compared with the oracle at its full size, in the launch configuration the
+benchmark times: every output element of every head (o and S_T), for the long-context workload
+the whole 65536-token sequence of all 96 heads, and for decode all 1000 in-place steps of the
+256 x 96 batch (o at every step, the state at the end).  Tolerance: max |x - ref| / max |ref|
+<= 2e-2 (bf16), 1e-4 (fp32), per output tensor; the per-head figure and the element-wise error
+are recorded (tests/helpers.check_parity) and printed at the end of the session.  Small
+adversarial and ragged cases compare every element too.
 """
 import numpy as np
 import pytest
@@ -12,29 +16,16 @@ import oracle
 import linear_attention_recurrence_forward_b200 as kda
 from linear_attention_recurrence_forward_b200.inputs import (PREFILL_CONFIGS, DECODE_CONFIG, make_config_inputs,
                                                              make_prefill_inputs, make_decode_inputs)
-from helpers import max_rel_err
+from helpers import max_rel_err, check_parity, error_stats, merge_stats, PARITY_LOG
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
+TOL_BF16, TOL_FP32 = 2e-2, 1e-4
+O_HEADS, S_HEADS = (0, 2), (0, 1)     # head axes of o [B, T, H, dv] and of states [B, H, dk, dv]
 
 
 def to_np(t):
     return t.detach().to("cpu", torch.float64).numpy()
-
-
-def head_slice(x, b, h):
-    return x[b:b + 1, :, h:h + 1].contiguous()
-
-
-def oracle_heads(inputs, heads):
-    """Oracle on the selected (b, h) heads, stacked along the head axis so they run in parallel."""
-    q, k, v, g, beta, S0 = inputs
-    idx_b = [b for b, _ in heads]
-    idx_h = [h for _, h in heads]
-    pick = lambda x: torch.stack([x[b, :, h] for b, h in zip(idx_b, idx_h)], dim=1)[None].contiguous()
-    s0 = None if S0 is None else torch.stack([S0[b, h] for b, h in zip(idx_b, idx_h)])[None].contiguous()
-    o_ref, ST_ref = oracle.forward(pick(q), pick(k), pick(v), pick(g), pick(beta), s0, nthreads=0)
-    return [(o_ref[:, :, j:j + 1], ST_ref[:, j:j + 1]) for j in range(len(heads))]
 
 
 @pytest.mark.parametrize("T", [64, 128, 191, 320, 1000])
@@ -55,8 +46,9 @@ def test_tc_matches_oracle(T, regime):
     torch.cuda.synchronize()
     assert kda.kda_get_device_status() == 0
     o_ref, ST_ref = oracle.forward(q, k, v, g, beta, S0, nthreads=0)
-    assert max_rel_err(to_np(o), o_ref) <= 2e-2
-    assert max_rel_err(to_np(ST), ST_ref) <= 2e-2
+    case = f"tc T={T} {regime}"
+    check_parity(case, "o", to_np(o), o_ref, TOL_BF16, O_HEADS)
+    check_parity(case, "S_T", to_np(ST), ST_ref, TOL_BF16, S_HEADS)
 
 
 def test_tc_agrees_with_fp32_simt_kernel():
@@ -76,8 +68,8 @@ def test_config_h32_t4k_full():
     torch.cuda.synchronize()
     assert kda.kda_get_device_status() == 0
     o_ref, ST_ref = oracle.forward(*inputs, nthreads=0)
-    assert max_rel_err(to_np(o), o_ref) <= 2e-2
-    assert max_rel_err(to_np(ST), ST_ref) <= 2e-2
+    check_parity(cfg.name, "o", to_np(o), o_ref, TOL_BF16, O_HEADS, TOL_BF16)
+    check_parity(cfg.name, "S_T", to_np(ST), ST_ref, TOL_BF16, S_HEADS, TOL_BF16)
 
 
 def test_config_small_fp32_full():
@@ -86,49 +78,77 @@ def test_config_small_fp32_full():
     o, ST = kda.kda_forward_chunked(*inputs)
     torch.cuda.synchronize()
     o_ref, ST_ref = oracle.forward(*inputs)
-    assert max_rel_err(to_np(o), o_ref) <= 1e-4
-    assert max_rel_err(to_np(ST), ST_ref) <= 1e-4
+    check_parity(cfg.name, "o", to_np(o), o_ref, TOL_FP32, O_HEADS, TOL_FP32)
+    check_parity(cfg.name, "S_T", to_np(ST), ST_ref, TOL_FP32, S_HEADS, TOL_FP32)
 
 
-def test_config_k3_b4_t8k_sampled_heads():
-    """The benchmark's K3 workload (B4 T8192 H96), launched whole; 8 heads checked end to end."""
+def test_config_k3_b4_t8k_every_head():
+    """The benchmark's K3 workload (B4 T8192 H96, S0 ~ N(0, 0.02^2), slow decay), launched whole as
+    the benchmark launches it: every element of o and S_T of all 384 heads against the oracle
+    (run one batch entry, i.e. 96 heads, at a time to bound host memory)."""
     cfg = PREFILL_CONFIGS["k3_b4_t8k"]
-    inputs = make_config_inputs(cfg, device=DEV)
-    o, ST = kda.kda_forward_chunked(*inputs)
+    q, k, v, g, beta, S0 = make_config_inputs(cfg, device=DEV)
+    o, ST = kda.kda_forward_chunked(q, k, v, g, beta, S0)
     torch.cuda.synchronize()
     assert kda.kda_get_device_status() == 0
     assert torch.isfinite(o).all() and torch.isfinite(ST).all()
-    heads = [(0, 0), (0, 95), (1, 17), (1, 48), (2, 63), (2, 5), (3, 94), (3, 31)]
-    for (b, h), (o_ref, ST_ref) in zip(heads, oracle_heads(inputs, heads)):
-        assert max_rel_err(to_np(head_slice(o, b, h)), o_ref) <= 2e-2, (b, h)
-        assert max_rel_err(to_np(ST[b:b + 1, h:h + 1]), ST_ref) <= 2e-2, (b, h)
+    so, ss = [], []
+    for b in range(cfg.B):
+        sl = lambda x: x[b:b + 1]
+        o_ref, ST_ref = oracle.forward(sl(q), sl(k), sl(v), sl(g), sl(beta), sl(S0), nthreads=0)
+        so.append(error_stats(to_np(sl(o)), o_ref, O_HEADS))
+        ss.append(error_stats(to_np(sl(ST)), ST_ref, S_HEADS))
+        del o_ref, ST_ref
+    for tensor, items in (("o", so), ("S_T", ss)):
+        s = merge_stats(items)
+        PARITY_LOG.append(dict(case=cfg.name, tensor=tensor, tol=TOL_BF16, **s))
+        assert s["rel"] <= TOL_BF16 and s["head_rel"] <= TOL_BF16, (tensor, s)
 
 
-def test_config_k3_t64k_prefix_and_final_state():
-    """B1 T65536 H96: o on the first 4096 tokens and the full-length S_T, for sampled heads."""
+def test_config_k3_t64k_every_head():
+    """B1 T65536 H96 (1024 chunks carried in sequence): o and the full-length S_T of all 96 heads
+    against the oracle; the 4096-token prefix of o is also reported on its own.  The oracle runs
+    24 heads at a time to bound host memory."""
     cfg = PREFILL_CONFIGS["k3_t64k"]
-    inputs = make_config_inputs(cfg, device=DEV)
-    o, ST = kda.kda_forward_chunked(*inputs)
+    q, k, v, g, beta, S0 = make_config_inputs(cfg, device=DEV)
+    o, ST = kda.kda_forward_chunked(q, k, v, g, beta, S0)
     torch.cuda.synchronize()
     assert kda.kda_get_device_status() == 0
-    heads = [(0, 0), (0, 41), (0, 77), (0, 95)]
-    for (b, h), (o_ref, ST_ref) in zip(heads, oracle_heads(inputs, heads)):
-        assert max_rel_err(to_np(head_slice(o, b, h)[:, :4096]), o_ref[:, :4096]) <= 2e-2, (b, h)
-        assert max_rel_err(to_np(head_slice(o, b, h)), o_ref) <= 2e-2, (b, h)
-        assert max_rel_err(to_np(ST[b:b + 1, h:h + 1]), ST_ref) <= 2e-2, (b, h)
+    assert torch.isfinite(o).all() and torch.isfinite(ST).all()
+    so, sp, ss = [], [], []
+    for h0 in range(0, cfg.H, 24):
+        sl = lambda x: x[:, :, h0:h0 + 24]
+        o_ref, ST_ref = oracle.forward(sl(q), sl(k), sl(v), sl(g), sl(beta), None, nthreads=0)
+        o_gpu = to_np(sl(o))
+        so.append(error_stats(o_gpu, o_ref, O_HEADS))
+        sp.append(error_stats(o_gpu[:, :4096], o_ref[:, :4096], O_HEADS))
+        ss.append(error_stats(to_np(ST[:, h0:h0 + 24]), ST_ref, S_HEADS))
+        del o_ref, ST_ref, o_gpu
+    for tensor, items in (("o", so), ("o[:4096]", sp), ("S_T", ss)):
+        s = merge_stats(items)
+        PARITY_LOG.append(dict(case=cfg.name, tensor=tensor, tol=TOL_BF16, **s))
+        assert s["rel"] <= TOL_BF16 and s["head_rel"] <= TOL_BF16, (tensor, s)
 
 
-def test_config_decode_full_batch():
-    """256 sequences x 96 heads, 128x128 fp32 states, updated in place: 3 steps, every element."""
+def test_config_decode_1000_steps_full_batch():
+    """256 sequences x 96 heads, 128x128 fp32 states updated in place for the workload's 1000
+    steps (fresh bf16 tokens each step, S = 0 at step 0): o of every step and the final state,
+    every element, against the oracle's own 1000 steps."""
     D = DECODE_CONFIG
     gen = torch.Generator(device=DEV)
     gen.manual_seed(D.seed)
     S = torch.zeros((D.batch, D.H, D.dk, D.dv), dtype=torch.float32, device=DEV)
     S_ref = np.zeros((D.batch, D.H, D.dk, D.dv))
-    for _ in range(3):
+    so = []
+    for step in range(D.steps):
         x = make_decode_inputs(D.batch, D.H, D.dk, D.dv, D.dtype, gen=gen, device=DEV)
         o = kda.kda_decode_step(*x, S)
         o_ref = oracle.decode_step(*x, S_ref, nthreads=0)
-        torch.cuda.synchronize()
-        assert max_rel_err(to_np(o), o_ref) <= 2e-2
-    assert max_rel_err(to_np(S), S_ref) <= 2e-2
+        s = error_stats(to_np(o), o_ref, (0, 1))
+        assert s["rel"] <= TOL_BF16, (step, s)
+        so.append(s)
+    assert kda.kda_get_device_status() == 0
+    s = merge_stats(so)
+    PARITY_LOG.append(dict(case=f"{D.name} x{D.steps}", tensor="o (all)", tol=TOL_BF16, **s))
+    assert s["head_rel"] <= TOL_BF16, s
+    check_parity(f"{D.name} x{D.steps}", "S", to_np(S), S_ref, TOL_BF16, S_HEADS, TOL_BF16)

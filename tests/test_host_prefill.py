@@ -93,6 +93,7 @@ def _pinned(t):
 @pytest.mark.parametrize("B,T,H,d,dtype,impl,s0", [
     (2, 5000, 3, 128, "bf16", "tcgen05", True),     # three segments per sequence, ragged last one
     (3, 2048, 2, 128, "bf16", "tcgen05", False),    # exactly one segment, zero initial state
+    (4, 5000, 2, 128, "bf16", "tcgen05", True),     # state slot b % 2 reused by b + 2, each with an S0 copy-in
     (1, 4097, 2, 128, "bf16", "auto", True),        # one token past two segments
     (2, 300, 2, 64, "fp32", "simt", True),          # the CUDA-core kernel
     (2, 4200, 1, 64, "bf16", "simt", False),

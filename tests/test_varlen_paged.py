@@ -143,21 +143,33 @@ def test_rows_outside_the_ranges_are_untouched(impl):
 
 @gpu
 @pytest.mark.parametrize("impl", ["tcgen05", "simt"])
-def test_invalid_offsets_are_reported_not_followed(impl):
+@pytest.mark.parametrize("fault", ["past_end", "overlap", "negative"])
+def test_invalid_offsets_are_reported_not_followed(impl, fault):
+    """Offsets that are not one valid layout (a range past the tokens, two overlapping ranges, a
+    negative start) are reported and no sequence is processed: every S_T is its S0 and no o row is
+    written, so no two CTAs ever write the same rows."""
     lengths = [100, 60, 80]
     q, k, v, g, beta, cu, S0 = packed_case(lengths, 2, 128, "bf16", seed=8)
     bad = cu.clone()
-    bad[3] = q.shape[0] + 50    # sequence 2 runs past the tokens
+    if fault == "past_end":
+        bad[3] = q.shape[0] + 50    # sequence 2 runs past the tokens
+    elif fault == "overlap":
+        bad[1], bad[2] = 120, 90    # sequence 1 is [120, 90) (backwards); 0 = [0, 120) and 2 = [90, 240) overlap
+    else:
+        bad[0] = -4
     assert kda.kda_get_device_status() == 0
-    o, ST = kda.kda_forward_varlen(q, k, v, g, beta, bad, S0, impl=impl)
+    o = torch.full((q.shape[0], 2, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    o, ST = kda.kda_forward_varlen(q, k, v, g, beta, bad, S0, o=o, impl=impl)
     assert kda.kda_get_device_status() == STATUS["KDA_ERR_INVALID_ARG"]
-    assert torch.equal(ST[2], S0[2])                     # processed as empty
-    for n in (0, 1):                                     # the others are still right
-        s0, s1 = int(bad[n]), int(bad[n + 1])
+    assert torch.equal(ST, S0)                           # every sequence processed as empty
+    assert bool((o == 7.0).all())                        # nothing written
+    o, ST = kda.kda_forward_varlen(q, k, v, g, beta, cu, S0, impl=impl)
+    assert kda.kda_get_device_status() == 0              # valid offsets: the word was cleared by the read
+    for n in range(3):
+        s0, s1 = int(cu[n]), int(cu[n + 1])
         o_ref, ST_ref = oracle.forward(*[x[s0:s1][None] for x in (q, k, v, g, beta)], S0[n:n + 1])
         assert max_rel_err(np64(o[s0:s1]), o_ref[0]) <= 2e-2
         assert max_rel_err(np64(ST[n]), ST_ref[0]) <= 2e-2
-    assert kda.kda_get_device_status() == 0              # the word was cleared by the read
 
 
 def decode_inputs(B, H, d, dtype, seed):
