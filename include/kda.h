@@ -24,7 +24,8 @@
  *   - All tensor pointers are DEVICE pointers owned by the caller (except in
  *     kda_forward_chunked_host, which takes HOST buffers and a caller-owned device
  *     workspace).  The library never allocates, frees or retains caller memory.  It owns one
- *     small static device status word per device (see kda_get_device_status).
+ *     small static device status word per device (see kda_get_device_status) and the fixed
+ *     scratch array of kda_forward_chunked_host_noalloc (KDA_NOALLOC_SCRATCH_BYTES per device).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
  *     stream).  A return of KDA_OK means the work was validated and enqueued.
  *   - Tensors are contiguous, row-major, with the layouts stated per function.
@@ -175,6 +176,69 @@ KDA_API int kda_forward_chunked_host(const void* q, const void* k, const void* v
  * outputs plus two states.  Returns 0 for an unsupported dtype or head size, H <= 0 or T < 0.
  */
 KDA_API size_t kda_forward_chunked_host_workspace(int T, int H, int dk, int dv, int dtype);
+
+/*
+ * KDA_NOALLOC_SCRATCH_BYTES -- size of the fixed device scratch array that
+ * kda_forward_chunked_host_noalloc stages its work through (32 MiB).  The library reserves it
+ * in the device memory of every GPU it is loaded on, when it is loaded, and holds it until the
+ * process exits.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/*
+ * kda_forward_chunked_host_noalloc -- kda_forward_chunked_host for callers that cannot allocate
+ * device memory.  (The pages describe no such entry point: it is an interface matter of this
+ * library, with no counterpart in the method.)
+ *
+ * Who needs it: a caller that holds only host arrays and reaches the library through a plain C
+ * foreign-function interface, with no CUDA allocator of its own to create the device workspace
+ * kda_forward_chunked_host asks for; or an engine whose device memory is all owned by a pool that
+ * forbids allocations outside it (and in which a cudaMalloc would also synchronise the device in
+ * the middle of its work).  This call allocates nothing, on the device or the host: it calls no
+ * cudaMalloc, cudaFree, stream or event creation, or any other allocating routine.  Instead it
+ * stages the work through one fixed scratch array of KDA_NOALLOC_SCRATCH_BYTES that the library
+ * reserves when it is loaded.
+ *
+ *   q, k, v, g, beta, S0, o, S_T : HOST buffers, with the layouts, dtypes, NULL rules and overlap
+ *              rules of kda_forward_chunked_host (S_T may be S0 itself).  Page-locked memory makes
+ *              the copies asynchronous.  With pageable memory the copies are staged by the driver
+ *              and the call blocks the host thread.  Inputs must stay unchanged, and outputs unread,
+ *              until the work on `stream` completes.
+ *   impl     : kda_impl, as for kda_forward_chunked_impl.
+ *
+ * Every step runs in order on `stream`: the inputs of one segment are copied in, the prefill runs
+ * on them, and o (and S_T after a sequence's last segment) is copied out.  A segment is one batch
+ * entry and the largest multiple of 64 tokens whose q, k, g, v, beta and o fit the scratch
+ * together with one fp32 state [H, dk, dv]: 192 tokens for H = 96 and bf16 d = 128.
+ * The state carried between the segments of a sequence stays in fp32 device memory, so o and S_T
+ * are bitwise those of kda_forward_chunked_host and kda_forward_chunked on the same values.  There
+ * is no overlap of copies with kernels: this entry point trades speed for needing no memory.
+ *
+ * Maximum size: the state of one batch entry plus 64 tokens of inputs and outputs (T tokens when
+ * T < 64) must fit the scratch: 256-byte-rounded H*dk*dv*4 + 3*n*dk*e + 2*n*dv*e + n*e bytes, with
+ * n = H * min(T, 64) and e = 2 (bf16) or 4 (fp32).  So H <= 227 at bf16 d = 128 and H <= 146 at
+ * fp32 d = 128.  Larger problems return KDA_ERR_UNSUPPORTED before anything is enqueued.
+ *
+ * Shared scratch: the array is one per device, shared by every call on that device, and it keeps
+ * the last call's contents.  Nothing in it needs to start at zero: a sequence without S0 starts
+ * from the zero state inside the kernel, and every byte a segment reads is first written by that
+ * same segment's copy-in.  Calls whose work overlaps on the GPU (on different streams, or on one
+ * stream from different host threads without ordering) race on the scratch and give undefined
+ * results: run them in order, on one stream.
+ *
+ * First call on a device: it looks up the device address of the scratch (cudaGetSymbolAddress,
+ * with that device current) and keeps it for later calls.  Make that first call before any
+ * stream capture on the device.
+ *
+ * Returns KDA_OK; KDA_ERR_INVALID_ARG or KDA_ERR_UNSUPPORTED (also: the problem does not fit the
+ * scratch, as above) before anything is enqueued, as kda_forward_chunked_host; KDA_ERR_CUDA if the
+ * scratch's address cannot be looked up, or if a copy or launch fails part-way (work already
+ * enqueued on `stream` still runs).
+ */
+KDA_API int kda_forward_chunked_host_noalloc(const void* q, const void* k, const void* v, const void* g,
+                                             const void* beta, const float* S0, void* o, float* S_T, int B,
+                                             int T, int H, int dk, int dv, int dtype, int impl,
+                                             struct CUstream_st* stream);
 
 /*
  * kda_decode_step -- one token for every (b, h), state updated in place.

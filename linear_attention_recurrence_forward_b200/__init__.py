@@ -26,6 +26,7 @@ __all__ = [
     "kda_forward_chunked",
     "kda_forward_chunked_states",
     "kda_forward_chunked_host",
+    "kda_forward_chunked_host_noalloc",
     "host_workspace_bytes",
     "kda_decode_step",
     "kda_forward_varlen",
@@ -83,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.kda_forward_chunked_states.restype = I
         L.kda_forward_chunked_host.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, ctypes.c_size_t, I, P]
         L.kda_forward_chunked_host.restype = I
+        L.kda_forward_chunked_host_noalloc.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P]
+        L.kda_forward_chunked_host_noalloc.restype = I
         L.kda_forward_chunked_host_workspace.argtypes = [I, I, I, I, I]
         L.kda_forward_chunked_host_workspace.restype = ctypes.c_size_t
         L.kda_state_compose.argtypes = [P, P, P, P, I, I, I, P]
@@ -224,6 +227,44 @@ def kda_forward_chunked_host(q, k, v, g, beta, S0=None, *, o=None, S_T=None, ret
             raise KdaError("kda_forward_chunked_host", rc)
         if own_workspace and stream is not None:
             workspace.record_stream(stream)   # not reused before the call's work on `stream` is done
+    return o, S_T
+
+
+def kda_forward_chunked_host_noalloc(q, k, v, g, beta, S0=None, *, o=None, S_T=None, return_state: bool = True,
+                                     impl: str = "auto", stream=None, device=None):
+    """kda_forward_chunked_host without a workspace: the library stages the work through its own fixed
+    device scratch (KDA_NOALLOC_SCRATCH_BYTES per device), so nothing is allocated on the device.
+    Host tensors in, host tensors out (outputs allocated here are pinned); o and S_T equal
+    kda_forward_chunked_host's bitwise.  Calls whose work overlaps on the GPU share the scratch and
+    race: keep them in order on one stream.  Read o and S_T after synchronizing `stream`.
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if dt not in DTYPE:
+        raise ValueError(f"unsupported dtype {dt}")
+    cpu = torch.device("cpu")
+    for name, t, shape in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("v", v, (B, T, H, dv)),
+                           ("g", g, (B, T, H, dk)), ("beta", beta, (B, T, H))):
+        _check(t, name, shape, dt, cpu)
+    if S0 is not None:
+        _check(S0, "S0", (B, H, dk, dv), torch.float32, cpu)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, pin_memory=True)
+    else:
+        _check(o, "o", (B, T, H, dv), dt, cpu)
+    if S_T is None and return_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, pin_memory=True)
+    elif S_T is not None:
+        _check(S_T, "S_T", (B, H, dk, dv), torch.float32, cpu)
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(device):
+        rc = lib().kda_forward_chunked_host_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                                                    _ptr(o), _ptr(S_T), B, T, H, dk, dv, DTYPE[dt], IMPL[impl],
+                                                    _stream_handle(stream))
+    if rc != 0:
+        raise KdaError("kda_forward_chunked_host_noalloc", rc)
     return o, S_T
 
 
