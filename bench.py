@@ -514,6 +514,40 @@ def run_ours(args):
     return 0
 
 
+def run_decode_only(args):
+    """Decode steps back to back on one GPU (profiling: consecutive launches of the decode kernel, so that
+    the state lines one launch leaves dirty in L2 are written back during the next)."""
+    import torch
+    import linear_attention_recurrence_forward_b200 as kda
+    from linear_attention_recurrence_forward_b200.inputs import make_decode_inputs
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    D = DECODE
+    gen = torch.Generator(device=str(dev))
+    gen.manual_seed(2000)
+    ring = [make_decode_inputs(D["batch"], D["H"], D["dk"], D["dv"], D["dtype"], gen=gen, device=str(dev))
+            for _ in range(DECODE_RING)]
+    S = torch.zeros((D["batch"], D["H"], D["dk"], D["dv"]), dtype=torch.float32, device=dev)
+    od = torch.empty((D["batch"], D["H"], D["dv"]), dtype=ring[0][0].dtype, device=dev)
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        kda.kda_decode_step(*ring[i % DECODE_RING], S, o=od, stream=stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(args.steps):
+        kda.kda_decode_step(*ring[i % DECODE_RING], S, o=od, stream=stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if kda.kda_get_device_status() != 0:
+        raise RuntimeError("device status after the decode steps")
+    ms = t0.elapsed_time(t1) / args.steps
+    db_ = decode_alg_bytes(D["batch"], D["H"], D["dk"], D["dv"])
+    print(json.dumps({"mode": "decode-only (profiling)", "workload": D["name"], "ms_per_step": ms,
+                      "alg_bytes_per_launch": db_, "achieved_gbs": db_ / (ms / 1e3) / 1e9}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -528,6 +562,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-states", action="store_true", help="skip the state-emission (every 512 tokens) timing")
     ap.add_argument("--no-long", action="store_true", help="skip the long-context (T = 65536) timing")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="profiling: run only decode steps back to back (no prefill between them) and print their "
+                         "timing; not the benchmark line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -538,6 +575,8 @@ def main():
         DECODE.update(batch=args.decode_batch, name=f"decode_b{args.decode_batch}_h{DECODE['H']}")
     if args.impl == "reference":
         return run_reference(args)
+    if args.decode_only:
+        return run_decode_only(args)
     return run_ours(args)
 
 

@@ -343,6 +343,30 @@ KDA_API int kda_state_compose(const float* M, const float* S_in, const float* N,
                               int dk, int dv, struct CUstream_st* stream);
 
 /*
+ * kda_output_correct -- correct the outputs of a segment that was run from a zero state, once the
+ * state it really starts from is known: o_out[b,t,h,:] = o_in[b,t,h,:] + S_in[b,h]^T C[b,t,h,:].
+ *
+ * Over a segment S_t = Phi_t S_in + S_t^0 (Phi_t = prod_{u<=t} (I - beta_u k_u k_u^T) Diag(exp g_u),
+ * S_t^0 the state from a zero start), so o_t = o_t^0 + S_in^T (Phi_t^T q_t).  The correction operand
+ * C_t = Phi_t^T q_t is the output of kda_forward_chunked on the same q, k, g, beta with v = 0 (dv = dk)
+ * and S0 = the identity; its S_T is the segment's map M (see kda_state_compose).  This is the one
+ * exchange step of KDA context parallelism (channel post on the K3 report (t.iss.one),
+ * infrastructure paragraph): a rank runs its segment before its incoming state is known, then
+ * applies this correction.
+ *
+ *   C      : [B, T, H, dk]  dtype
+ *   S_in   : [B, H, dk, dv] fp32
+ *   o_in   : [B, T, H, dv]  dtype (the zero-start outputs)
+ *   o_out  : [B, T, H, dv]  dtype output (bf16 rounded to nearest even); may be o_in itself
+ *
+ * bf16 with dk = dv = 128 runs on the tensor core (S_in rounded to bf16 as the product's operand,
+ * fp32 accumulation); other shapes and fp32 on CUDA cores in fp32.  T == 0 does nothing.  Returns
+ * KDA_OK or a negative kda_status (nothing enqueued on error).
+ */
+KDA_API int kda_output_correct(const void* C, const float* S_in, const void* o_in, void* o_out, int B, int T, int H,
+                               int dk, int dv, int dtype, struct CUstream_st* stream);
+
+/*
  * kda_get_device_status -- synchronise `stream`, then return and clear the status word
  * of the current device: KDA_OK, KDA_ERR_TIMEOUT (a kernel's bounded wait gave up; its
  * outputs are then undefined), KDA_ERR_INVALID_ARG (a kernel found an out-of-range device

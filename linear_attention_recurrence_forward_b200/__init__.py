@@ -33,6 +33,7 @@ __all__ = [
     "kda_forward_chunked_fused",
     "kda_decode_step_paged",
     "kda_state_compose",
+    "kda_output_correct",
     "kda_get_device_status",
     "kda_status_string",
     "kda_debug_set_wait_fault",
@@ -90,6 +91,8 @@ def lib() -> ctypes.CDLL:
         L.kda_forward_chunked_host_workspace.restype = ctypes.c_size_t
         L.kda_state_compose.argtypes = [P, P, P, P, I, I, I, P]
         L.kda_state_compose.restype = I
+        L.kda_output_correct.argtypes = [P, P, P, P, I, I, I, I, I, I, P]
+        L.kda_output_correct.restype = I
         L.kda_forward_chunked_fused.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P]
         L.kda_forward_chunked_fused.restype = I
         L.kda_forward_varlen.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P]
@@ -446,6 +449,31 @@ def kda_state_compose(M, S, N=None, *, out=None, stream=None):
         rc = lib().kda_state_compose(_ptr(M), _ptr(S), _ptr(N), _ptr(out), count, dk, dv, _stream_handle(stream))
     if rc != 0:
         raise KdaError("kda_state_compose", rc)
+    return out
+
+
+def kda_output_correct(C, S_in, o_in, *, out=None, stream=None):
+    """out = o_in + per token S_in^T C: C [B, T, H, dk], o_in [B, T, H, dv] (same dtype) and S_in
+    [B, H, dk, dv] fp32 CUDA tensors.  out may be o_in itself.  The output correction of a segment
+    run from a zero state (context parallelism): C is the output of the same segment with v = 0 and
+    S0 = I."""
+    B, T, H, dk = C.shape
+    dv = o_in.shape[-1]
+    dev, dt = C.device, C.dtype
+    if dt not in DTYPE:
+        raise ValueError(f"unsupported dtype {dt}")
+    _check(C, "C", (B, T, H, dk), dt, dev)
+    _check(o_in, "o_in", (B, T, H, dv), dt, dev)
+    _check(S_in, "S_in", (B, H, dk, dv), torch.float32, dev)
+    if out is None:
+        out = torch.empty_like(o_in)
+    else:
+        _check(out, "out", (B, T, H, dv), dt, dev)
+    with torch.cuda.device(dev):
+        rc = lib().kda_output_correct(_ptr(C), _ptr(S_in), _ptr(o_in), _ptr(out), B, T, H, dk, dv, DTYPE[dt],
+                                      _stream_handle(stream))
+    if rc != 0:
+        raise KdaError("kda_output_correct", rc)
     return out
 
 

@@ -435,6 +435,31 @@ int kda_state_compose(const float* M, const float* S_in, const float* N, float* 
     return kda::launch_state_compose(M, S_in, N, S_out, count, dk, dv, stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+int kda_output_correct(const void* C, const float* S_in, const void* o_in, void* o_out, int B, int T, int H, int dk,
+                       int dv, int dtype, struct CUstream_st* stream) {
+    if (B <= 0 || H <= 0 || T < 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_FP32) return KDA_ERR_UNSUPPORTED;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if ((double)B * (double)T * (double)H * (double)(dk > dv ? dk : dv) > 9.0e15) return KDA_ERR_INVALID_ARG;
+    if (T == 0) return KDA_OK;
+    if (!C || !S_in || !o_in || !o_out) return KDA_ERR_INVALID_ARG;
+    const void* ptrs[] = {C, S_in, o_in, o_out};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+    const size_t es = elem_size(dtype);
+    const size_t n_tok = (size_t)B * T * H;
+    const Range ro = range_of(o_out, n_tok * dv * es);
+    const Range rc = range_of(C, n_tok * dk * es);
+    const Range rs = range_of(S_in, (size_t)B * H * dk * dv * sizeof(float));
+    // o_out may be o_in itself (in place); no other overlap
+    if (overlaps(ro, rc) || overlaps(ro, rs)) return KDA_ERR_INVALID_ARG;
+    if (o_out != o_in && overlaps(ro, range_of(o_in, n_tok * dv * es))) return KDA_ERR_INVALID_ARG;
+    int* status = status_word_for_current_device();
+    if (!status) return KDA_ERR_CUDA;
+    return kda::launch_output_correct(C, S_in, o_in, o_out, B, T, H, dk, dv, dtype, status, g_timeout_ns.load(),
+                                      stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 int kda_get_device_status(struct CUstream_st* stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
     int* addr = status_word_for_current_device();

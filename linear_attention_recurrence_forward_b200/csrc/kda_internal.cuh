@@ -61,6 +61,12 @@ bool prefill_tc_supports(const PrefillArgs& a);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_state_compose(const float* M, const float* S, const float* N, float* out, int count, int dk,
                                  int dv, cudaStream_t s);
+// o_out = o_in + per token S^T C (kda_output_correct; arguments validated by the caller)
+cudaError_t launch_output_correct(const void* C, const float* S, const void* o_in, void* o_out, int B, int T, int H,
+                                  int dk, int dv, int dtype, int* status, unsigned long long timeout_ns,
+                                  cudaStream_t s);
+// The driver's cuTensorMapEncodeTiled (looked up once), or null.
+void* tensor_map_encoder();
 
 // Element loads/stores for the two input dtypes.
 __device__ __forceinline__ float load_elem(const float* p, size_t i) { return p[i]; }

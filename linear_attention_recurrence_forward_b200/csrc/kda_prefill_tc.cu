@@ -35,7 +35,8 @@
 //                      T, P, Kb tiles.
 //   serial warps 8..15 per chunk: MMA3 [Qt;Kt] S -> Y = V - Kt S -> MMA4 U = T Y ->
 //                      MMA5 O = Qt S + P U, MMA6 S += Kb^T U (state decayed in TMEM first)
-//                      -> O to global, S to bf16 for the next chunk.
+//                      -> O to global, S to bf16 for the next chunk.  One thread issues the
+//                      products, another the O store and the v loads.
 // All tcgen05 products are M = 128: products with 64 meaningful rows read 64 further rows
 // of other valid shared memory into TMEM lanes that are never read.
 #include <cudaTypedefs.h>
@@ -151,27 +152,6 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
         "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
         : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
     return d;
-}
-
-// Byte offset of K step kk (16 elements) inside an operand tile: K-major tiles advance 32 B
-// inside a 128-byte swizzle row and jump to the next 64-column atom every 4 steps; MN-major
-// tiles advance 16 rows (2048 B).
-template <bool MN, uint32_t ATOM>
-__device__ __forceinline__ constexpr uint32_t kstep_off(int kk) {
-    return MN ? (uint32_t)kk * 2048u : (uint32_t)(kk >> 2) * ATOM + (uint32_t)(kk & 3) * 32u;
-}
-
-// Issue D (+)= A * B over K = 16 * KSTEPS from one thread.  Descriptors are built once and
-// advanced by constant offsets (the start-address field is the low 14 bits, in 16-byte units).
-template <int KSTEPS, bool A_MN, uint32_t A_ATOM, bool B_MN, uint32_t B_ATOM>
-__device__ __forceinline__ void issue_mma(uint32_t d_tmem, uint32_t a_base, uint32_t b_base, uint32_t idesc,
-                                          bool accumulate) {
-    const uint64_t ad = smem_desc_sw128(a_base, A_MN ? A_ATOM : 16u, 1024u);
-    const uint64_t bd = smem_desc_sw128(b_base, B_MN ? B_ATOM : 16u, 1024u);
-#pragma unroll
-    for (int kk = 0; kk < KSTEPS; ++kk)
-        mma_bf16(d_tmem, ad + (kstep_off<A_MN, A_ATOM>(kk) >> 4), bd + (kstep_off<B_MN, B_ATOM>(kk) >> 4), idesc,
-                 (kk > 0 || accumulate) ? 1u : 0u);
 }
 
 // Warp-level bf16 tensor-core tile D(16x8) += A(16x16, row-major) * B(16x8, column-major), fp32
@@ -754,8 +734,11 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     } else {
         // ====================================================================== serial group
         const int stid = tid - kPrepThreads;                // 0..255
-        int pending = -1;                                   // chunk whose v load is in flight
-        int pending_qk = -1;                                // last chunk whose q,k loads this leader issued
+        // Two single-thread roles: the leader (stid 0) issues the tensor-core products and the q, k loads;
+        // the I/O thread (stid 32) stores O and loads the next v, so that the wait for the O store to
+        // have read its staging tile never holds up the next chunk's MMA3.
+        int pending = -1;                                   // I/O thread: chunk whose v load is in flight
+        int pending_qk = -1;                                // leader: last chunk whose q,k loads it issued
         // Once the prep group has published chunk c's operand tiles (bar_kq): MMA3 = [Qt0;Kt0;Qt1;Kt1] S
         // and the raw q, k of chunk c+1 into the buffers the prep group has finished reading.
         auto issue_for_chunk = [&](int c) {
@@ -787,7 +770,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             for (int j = 0; j < 64; j += 8)
                 *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_offset(i, cb0 + j, 16384)) = pack8(r + j);
         }
-        if (stid == 0 && nchunks > 0) { load_v(0); pending = 0; }
+        if (stid == 32 && nchunks > 0) { load_v(0); pending = 0; }
         fence_proxy_async_smem();
         tc_fence_before_sync();
         named_bar_sync(kBarSerial, kSerialThreads);
@@ -806,7 +789,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc_fence_after_sync();
             ok = named_bar_and(kBarSerial, kSerialThreads, ok);
             if (!ok) break;
-            if (stid == 0) pending = -1;
+            if (stid == 32) pending = -1;
             if (quarter & 1) {
                 const int tj = 32 * (quarter >> 1) + lane;
                 float ks[64];
@@ -921,7 +904,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             fence_proxy_async_smem();
             tc_fence_before_sync();
             named_bar_sync(kBarSerial, kSerialThreads);
-            if (stid == 0) {
+            if (stid == 32) {
                 // rows past the tensor's T are clipped by the tensor map
                 if (!row_stores) {
                     tma_store_4d(&tm_o, sm + OFF_V, 0, h, tok0 + t0, bmap);
@@ -932,17 +915,21 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     bulk_wait_read_all();   // the staged O is read: the next v may land on it
                     load_v(chunk + 1);
                     pending = chunk + 1;
-                    ok = mbar_wait(&bar_kq, par ^ 1u, p.timeout_ns);
-                    if (ok) issue_for_chunk(chunk + 1);
                 }
+            }
+            if (stid == 0 && chunk + 1 < nchunks) {
+                ok = mbar_wait(&bar_kq, par ^ 1u, p.timeout_ns);
+                if (ok) issue_for_chunk(chunk + 1);
             }
         }
         if (!ok && stid == 0) report_status(p.status, KDA_ERR_TIMEOUT);
-        if (stid == 0) {
+        if (stid == 32) {
             bulk_wait_all();
+            if (pending >= 0) (void)mbar_wait(&bar_v, (uint32_t)(pending & 1), p.timeout_ns);
+        }
+        if (stid == 0) {
             mma_commit(&bar_drain_s);
             if (!mbar_wait(&bar_drain_s, 0, p.timeout_ns)) report_status(p.status, KDA_ERR_TIMEOUT);
-            if (pending >= 0) (void)mbar_wait(&bar_v, (uint32_t)(pending & 1), p.timeout_ns);
             if (pending_qk >= 0) (void)mbar_wait(&bar_qk, (uint32_t)(pending_qk & 1), p.timeout_ns);
         }
         named_bar_sync(kBarSerial, kSerialThreads);
@@ -965,16 +952,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 // ------------------------------------------------------------------ host side
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-    });
-    return fn;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
 }
 
 // [B, T, H, 128] bf16 viewed as a 4-D tensor (d, H, T, B); box = 64 channels x 1 head x 64 tokens.
@@ -993,6 +971,19 @@ bool make_map(CUtensorMap* m, const void* ptr, int B, int T, int H) {
 }
 
 }  // namespace
+
+void* tensor_map_encoder() {
+    static void* fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = f;
+    });
+    return fn;
+}
 
 bool prefill_tc_supports(const PrefillArgs& a) {
     return a.dtype == KDA_DTYPE_BF16 && a.dk == kD && a.dv == kD;

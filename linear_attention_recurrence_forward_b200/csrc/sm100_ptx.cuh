@@ -54,7 +54,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 // of wall time (returns false).  Never traps, never spins forever.  The first test is inline;
 // the timed retry loop is one out-of-line copy, which keeps the callers' loops (and their
 // instruction-cache footprint) smaller.
-__device__ __noinline__ bool mbar_wait_slow(uint32_t a, uint32_t parity, uint64_t timeout_ns) {
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t a, uint32_t parity, uint64_t timeout_ns) {
     const uint64_t t0 = global_timer_ns();
     for (;;) {
 #pragma unroll 1
@@ -193,6 +193,27 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                      smem_u32(bar))
                  : "memory");
+}
+
+// Byte offset of K step kk (16 elements) inside an operand tile: K-major tiles advance 32 B
+// inside a 128-byte swizzle row and jump to the next 64-column atom every 4 steps; MN-major
+// tiles advance 16 rows (2048 B).
+template <bool MN, uint32_t ATOM>
+__device__ __forceinline__ constexpr uint32_t kstep_off(int kk) {
+    return MN ? (uint32_t)kk * 2048u : (uint32_t)(kk >> 2) * ATOM + (uint32_t)(kk & 3) * 32u;
+}
+
+// Issue D (+)= A * B over K = 16 * KSTEPS from one thread.  Descriptors are built once and
+// advanced by constant offsets (the start-address field is the low 14 bits, in 16-byte units).
+template <int KSTEPS, bool A_MN, uint32_t A_ATOM, bool B_MN, uint32_t B_ATOM>
+__device__ __forceinline__ void issue_mma(uint32_t d_tmem, uint32_t a_base, uint32_t b_base, uint32_t idesc,
+                                          bool accumulate) {
+    const uint64_t ad = smem_desc_sw128(a_base, A_MN ? A_ATOM : 16u, 1024u);
+    const uint64_t bd = smem_desc_sw128(b_base, B_MN ? B_ATOM : 16u, 1024u);
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk)
+        mma_bf16(d_tmem, ad + (kstep_off<A_MN, A_ATOM>(kk) >> 4), bd + (kstep_off<B_MN, B_ATOM>(kk) >> 4), idesc,
+                 (kk > 0 || accumulate) ? 1u : 0u);
 }
 
 // TMEM -> registers: this warp's 32 lanes, 16 consecutive 32-bit columns.

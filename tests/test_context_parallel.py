@@ -1,5 +1,5 @@
 """KDA context parallelism: a batch of sequences split along T over ranks, only the fixed-size
-state maps exchanged.
+state maps exchanged, each rank's outputs corrected once its incoming state is known.
 
 CPU: the orchestration with an fp64 stand-in for the per-segment kernels (the oracle), both
 as ranks emulated in one process and as real gloo ranks (world sizes 2 and 3, ragged
@@ -35,6 +35,9 @@ class OracleOps:
     def compose(self, M, S, N):
         return torch.matmul(M, S) + N
 
+    def correct(self, C, S, o0):
+        return o0 + torch.einsum("bthi,bhij->bthj", C, S)
+
 
 def split_points(T, world, seed):
     rng = np.random.default_rng(seed)
@@ -58,7 +61,8 @@ def emulate(xs, S0, bounds, ops):
     outs, S_end = [first[0][2]], first[0][3]
     for r in range(1, world):
         S_in = cp.incoming_state(Ms, Ns, r, ops)
-        o, S_end = cp.rank_finish(S_in, *segs[r], ops=ops)
+        M, N, o0, _, C = first[r]
+        o, S_end = cp.rank_finish(S_in, o0, C, M, N, ops=ops)
         outs.append(o)
     return torch.cat(outs, dim=1), S_end
 
@@ -81,6 +85,23 @@ def test_segment_map_is_the_affine_map():
     # plausible slips do not pass: the transposed map, or dropping N
     assert max_rel_err((torch.matmul(M.transpose(-1, -2), S0) + N).numpy(), ST) > 1e-3
     assert max_rel_err(torch.matmul(M, S0).numpy(), ST) > 1e-3
+
+
+def test_correction_operand_is_the_state_map_read_out():
+    """C_t from the v = 0, S0 = I run satisfies o_t = o0_t + S^T C_t for any start state S, token by
+    token, and its final state is the map M (fp64 stand-in)."""
+    xs, S0 = problem(T=70, seed=9)
+    o0, N, C, M = cp.segment_pass(*xs, ops=OracleOps())
+    o_ref, ST_ref = oracle.forward(*xs, S0)
+    o = o0 + torch.einsum("bthi,bhij->bthj", C, S0)
+    assert max_rel_err(o.numpy(), o_ref) < 1e-12
+    assert max_rel_err((torch.matmul(M, S0) + N).numpy(), ST_ref) < 1e-12
+    # plausible slips do not pass: the correction dropped, or the segment's final map used for every
+    # token instead of the map up to that token
+    assert max_rel_err(o0.numpy(), o_ref) > 1e-3
+    q = xs[0]
+    o_end = o0 + torch.einsum("bthi,bhij->bthj", q, torch.matmul(M, S0))
+    assert max_rel_err(o_end.numpy(), o_ref) > 1e-3
 
 
 def _rank_main(rank, world, port, bounds, out):
@@ -163,13 +184,53 @@ def test_compose_kernel_matches_a_cpu_matmul(dk, dv):
     assert max_rel_err(kda.kda_state_compose(M, S).double().cpu().numpy(), ref0) < 1e-5
 
 
+def test_output_correct_rejects_bad_arguments(L):
+    C, S, Oi, Oo = (BASE + i * SZ for i in range(4))
+    f = L.kda_output_correct
+    assert f(C, S, Oi, Oo, 0, 64, 2, 128, 128, 0, None) == INVALID
+    assert f(C, S, Oi, Oo, 1, -1, 2, 128, 128, 0, None) == INVALID
+    assert f(C, S, Oi, Oo, 1, 64, 2, 96, 128, 0, None) == UNSUPPORTED
+    assert f(C, S, Oi, Oo, 1, 64, 2, 128, 128, 5, None) == UNSUPPORTED
+    assert f(None, S, Oi, Oo, 1, 64, 2, 128, 128, 0, None) == INVALID
+    assert f(C + 8, S, Oi, Oo, 1, 64, 2, 128, 128, 0, None) == MISALIGNED
+    assert f(C, S, Oi, C + 4096, 1, 64, 2, 128, 128, 0, None) == INVALID    # out inside C
+    assert f(C, S, Oi, Oi + 4096, 1, 64, 2, 128, 128, 0, None) == INVALID   # out partly over o_in
+    assert f(C, S, Oi, Oo, 1, 0, 2, 128, 128, 0, None) == OK                # no tokens: nothing to do
+
+
 @pytest.mark.gpu
-@pytest.mark.parametrize("dtype,world,T", [("bf16", 2, 1000), ("bf16", 4, 2100), ("fp32", 3, 400)])
-def test_context_parallel_steps_on_one_gpu(dtype, world, T):
+@pytest.mark.parametrize("dtype,dk,dv,T", [("bf16", 128, 128, 300), ("bf16", 128, 128, 128), ("bf16", 64, 128, 77),
+                                           ("fp32", 64, 64, 100), ("fp32", 128, 128, 33)])
+def test_output_correct_kernel_matches_a_cpu_product(dtype, dk, dv, T):
+    from linear_attention_recurrence_forward_b200.inputs import torch_dtype
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(T + dk)
+    dt = torch_dtype(dtype)
+    C = (torch.randn((2, T, 3, dk), generator=gen, device="cuda") * 0.3).to(dt)
+    o0 = torch.randn((2, T, 3, dv), generator=gen, device="cuda").to(dt)
+    S = torch.randn((2, 3, dk, dv), generator=gen, device="cuda") * 0.2
+    ref = (o0.double().cpu() + torch.einsum("bthi,bhij->bthj", C.double().cpu(), S.double().cpu())).numpy()
+    out = kda.kda_output_correct(C, S, o0)
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    tol = 2e-2 if dtype == "bf16" else 1e-5
+    assert max_rel_err(out.double().cpu().numpy(), ref) < tol
+    # in place over o_in
+    o1 = o0.clone()
+    kda.kda_output_correct(C, S, o1, out=o1)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, out)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype,world,T,zg_mean", [("bf16", 2, 1000, -8.0), ("bf16", 4, 2100, -8.0),
+                                                   ("bf16", 3, 2000, 0.0), ("fp32", 3, 400, -8.0)])
+def test_context_parallel_steps_on_one_gpu(dtype, world, T, zg_mean):
     from linear_attention_recurrence_forward_b200.inputs import make_prefill_inputs
     d = 128 if dtype == "bf16" else 64
-    # slow decay (z ~ N(-8, 1), g ~ -2e-3), so the composed states matter
-    q, k, v, g, beta, S0 = make_prefill_inputs(2, T, 3, d, d, dtype, seed=5, s0_std=0.05, zg_mean=-8.0,
+    # slow decay (z ~ N(-8, 1), g ~ -2e-3), so the composed states matter; and the recipe's decay
+    # (z ~ N(0, 1)), under which the maps M are far from the identity
+    q, k, v, g, beta, S0 = make_prefill_inputs(2, T, 3, d, d, dtype, seed=5, s0_std=0.05, zg_mean=zg_mean,
                                                device="cuda")
     bounds = [0] + [(T * r) // world // 64 * 64 + 17 * r for r in range(1, world)] + [T]
     o, ST = emulate([q, k, v, g, beta], S0, bounds, cp.CudaOps())
