@@ -199,8 +199,8 @@ def test_output_correct_rejects_bad_arguments(L):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("dtype,dk,dv,T", [("bf16", 128, 128, 300), ("bf16", 128, 128, 128), ("bf16", 64, 128, 77),
-                                           ("fp32", 64, 64, 100), ("fp32", 128, 128, 33)])
+@pytest.mark.parametrize("dtype,dk,dv,T", [("bf16", 128, 128, 300), ("bf16", 128, 128, 128), ("bf16", 128, 128, 1),
+                                           ("bf16", 64, 128, 77), ("fp32", 64, 64, 100), ("fp32", 128, 128, 33)])
 def test_output_correct_kernel_matches_a_cpu_product(dtype, dk, dv, T):
     from linear_attention_recurrence_forward_b200.inputs import torch_dtype
     gen = torch.Generator(device="cuda")
@@ -241,3 +241,33 @@ def test_context_parallel_steps_on_one_gpu(dtype, world, T, zg_mean):
     eo = max_rel_err(o.double().cpu().numpy(), o_ref)
     es = max_rel_err(ST.double().cpu().numpy(), ST_ref)
     assert eo <= tol and es <= tol, (eo, es)
+
+
+def _nccl_rank_main(rank, world, port, out):
+    """One rank of the NCCL path on its own GPU (context_parallel_forward with the CUDA kernels)."""
+    from datetime import timedelta
+    from linear_attention_recurrence_forward_b200.inputs import make_prefill_inputs
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    torch.cuda.set_device(rank)
+    dist.init_process_group("nccl", rank=rank, world_size=world, timeout=timedelta(seconds=60),
+                            device_id=torch.device("cuda", rank))
+    try:
+        q, k, v, g, beta, S0 = make_prefill_inputs(2, 500, 3, 128, 128, "bf16", seed=21, s0_std=0.05, device="cuda")
+        o, final = cp.context_parallel_forward(q, k, v, g, beta, S0=S0)
+        o_ref, ST_ref = kda.kda_forward_chunked(q, k, v, g, beta, S0)
+        torch.cuda.synchronize()
+        out[rank] = (bool(torch.equal(o, o_ref)), bool(torch.equal(final, ST_ref)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.gpu
+def test_nccl_path_on_one_gpu():
+    """context_parallel_forward over a one-rank NCCL group: the collectives run on device tensors and the
+    result equals the plain prefill bitwise (rank 0 runs its segment for real).  The exchange between
+    several GPUs is covered by the gloo ranks and the emulated GPU ranks above; one GPU is all a run has."""
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    port = 29950 + (os.getpid() % 40)
+    mp.start_processes(_nccl_rank_main, args=(1, port, out), nprocs=1, join=True, start_method="spawn")
+    assert out[0] == (True, True)
