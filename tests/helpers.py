@@ -3,7 +3,7 @@ import numpy as np
 
 # Every parity comparison that goes through check_parity() is recorded here and printed as a
 # table at the end of the pytest session (tests/conftest.py), so a run's log carries the
-# measured errors next to the pass/fail verdict.
+# measured errors next to the pass/fail result.
 PARITY_LOG = []
 
 
