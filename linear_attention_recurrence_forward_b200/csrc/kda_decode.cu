@@ -7,12 +7,15 @@
 // token; the same page (item D17, quiz Q5) is why it is memory-bound: every state
 // element is read and written once for ~7 flops.
 //
-// Design: one CTA of 256 threads per state.  Lanes run along the dv columns with 16-byte
-// vectors, so each warp instruction reads or writes whole contiguous rows (coalesced,
-// 512 B per warp); the state stays in registers between the read and the write (one
-// pass, no re-read).  Column sums over dk use warp shuffles (when a warp covers several
-// rows) and one shared-memory step across warps.  Loads/stores use the evict-first
-// streaming hints: a state is touched exactly once per step.
+// Design: the update is independent per value column (u_j and o_j need column j of the state and
+// the scalar k . q only), so a state is split over CTAs by columns: one CTA of 256 threads per
+// (state, 64-column slice), with no exchange between the slices.  That keeps 32 state values per
+// thread, so several CTAs share an SM and one CTA's reductions overlap the others' loads and
+// stores.  Lanes run along the columns with 16-byte vectors, so each warp instruction reads or
+// writes whole contiguous row segments (coalesced); the state stays in registers between the
+// read and the write (one pass, no re-read).  Column sums over dk use warp shuffles and one
+// shared-memory step across warps.  Loads/stores use the evict-first streaming hints: a state
+// is touched exactly once per step.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -20,12 +23,17 @@ namespace {
 
 constexpr int kDecodeThreads = 256;
 
+constexpr int kSliceCols = 64;   // state columns per CTA
+
+// DV: the state's columns (row stride); DVC: the columns of one CTA's slice
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kDecodeThreads)
 kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                   const Tin* __restrict__ g, const Tin* __restrict__ beta, float* __restrict__ S,
                   Tin* __restrict__ o, int H, const int* __restrict__ slots, int n_slots, int* status) {
-    constexpr int LPR = DV / 4;                    // threads per state row (float4 each)
+    constexpr int DVC = DV < kSliceCols ? DV : kSliceCols;
+    constexpr int NSL = DV / DVC;                  // slices per state
+    constexpr int LPR = DVC / 4;                   // threads per state row segment (float4 each)
     constexpr int RPP = kDecodeThreads / LPR;      // rows covered per pass
     constexpr int RPT = DK / RPP;                  // rows per thread
     constexpr int WPR = 32 / LPR;                  // rows per warp instruction (1 or 2)
@@ -39,7 +47,8 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
     const int c4 = tid % LPR, rg = tid / LPR;
-    const size_t bh = blockIdx.x;
+    const size_t bh = blockIdx.x / NSL;
+    const int col0 = (int)(blockIdx.x % NSL) * DVC;   // first column of this CTA's slice
     size_t sidx = bh;   // state of this (b, h): S[b, h], or S[slots[b], h] of a pool
     if (slots) {
         const int sl = slots[bh / H];
@@ -50,12 +59,13 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
         }
         sidx = (size_t)sl * H + bh % H;
     }
-    float4* Sv = reinterpret_cast<float4*>(S + sidx * DK * DV);
+    float4* Sv = reinterpret_cast<float4*>(S + sidx * DK * DV + col0);
+    constexpr int RS = DV / 4;                     // float4s per full state row
 
     // Issue the state loads first: 16 B per thread per row, all independent.
     float4 s[RPT];
 #pragma unroll
-    for (int j = 0; j < RPT; ++j) s[j] = __ldcs(Sv + (size_t)(rg + j * RPP) * LPR + c4);
+    for (int j = 0; j < RPT; ++j) s[j] = __ldcs(Sv + (size_t)(rg + j * RPP) * RS + c4);
 
     if (tid < DK) {
         qs[tid] = load_elem(q, bh * DK + tid);
@@ -101,7 +111,7 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
                 b.x += tb.x; b.y += tb.y; b.z += tb.z; b.w += tb.w;
             }
             const float bt = load_elem(beta, bh);
-            const size_t vo = bh * DV + 4 * lane;
+            const size_t vo = bh * DV + col0 + 4 * lane;
             float4 u;
             u.x = bt * (load_elem(v, vo + 0) - a.x);
             u.y = bt * (load_elem(v, vo + 1) - a.y);
@@ -121,13 +131,14 @@ kda_decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Ti
     for (int j = 0; j < RPT; ++j) {
         const float kr = ks[rg + j * RPP];
         s[j].x += kr * u.x; s[j].y += kr * u.y; s[j].z += kr * u.z; s[j].w += kr * u.w;
-        __stcs(Sv + (size_t)(rg + j * RPP) * LPR + c4, s[j]);
+        __stcs(Sv + (size_t)(rg + j * RPP) * RS + c4, s[j]);
     }
 }
 
 template <typename Tin, int DK, int DV>
 cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t s) {
-    const unsigned grid = (unsigned)((size_t)a.B * a.H);
+    constexpr int nsl = DV < kSliceCols ? 1 : DV / kSliceCols;
+    const unsigned grid = (unsigned)((size_t)a.B * a.H * nsl);
     kda_decode_kernel<Tin, DK, DV><<<grid, kDecodeThreads, 0, s>>>(
         static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
         static_cast<const Tin*>(a.g), static_cast<const Tin*>(a.beta), a.S, static_cast<Tin*>(a.o), a.H, a.slots,
