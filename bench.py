@@ -33,6 +33,8 @@ METRIC = "KDA prefill tokens/s (K3 shape, H=96, d=128) and decode states/s; % of
 PREFILL = dict(name="k3_b4_t8k", B=4, T=8192, H=96, dk=128, dv=128, dtype="bf16", s0_std=0.02, zg_mean=-2.0)
 DECODE = dict(name="decode_b256_h96", batch=256, H=96, dk=128, dv=128, dtype="bf16")
 LONG = dict(name="k3_t64k", B=1, T=65536, H=96, dk=128, dv=128, dtype="bf16")
+# the recorded ncu traffic (profiles/) is per launch of these two workloads
+DEFAULT_PREFILL_NAME, DEFAULT_DECODE_NAME = PREFILL["name"], DECODE["name"]
 DECODE_RING = 8
 
 
@@ -492,14 +494,15 @@ def run_ours(args):
                    "decode_batch": D["batch"], "l2": "inputs larger than L2 (4.1 GB prefill, 1.6 GB decode state)",
                    "parallelism": f"replicas x{world} (independent batches, no collective)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": recorded_traffic(impl_tag),
+                     "frac": achieved / peak,
+                     "traffic": recorded_traffic(impl_tag) if P["name"] == DEFAULT_PREFILL_NAME else None,
                      "kernel": impl_tag, "alg_bytes_per_launch": pb, "launch_ms": prefill_launch_ms,
                      "peak_kind": peak_kind, "tensor": tensor_line},
         "decode": {"states_per_s": decode_states_per_s, "tokens_per_s": decode_states_per_s / D["H"],
                    "ms_per_step": decode_launch_ms,
                    "roofline": {"bound": "hbm", "achieved": dec_achieved, "peak": peak, "unit": "GB/s",
                                 "frac": dec_achieved / peak, "alg_bytes_per_launch": db_,
-                                "traffic": recorded_traffic("decode")}},
+                                "traffic": recorded_traffic("decode") if D["name"] == DEFAULT_DECODE_NAME else None}},
         "long_context": long_line,
         "state_emission": states_line,
         "fused_prologue": fused_line,
@@ -559,6 +562,8 @@ def main():
     ap.add_argument("--prefill-shape", default=None, metavar="B,T,H",
                     help="override the prefill workload (profiling small cases); the line is then not the headline")
     ap.add_argument("--decode-batch", type=int, default=None, help="override the decode batch (profiling)")
+    ap.add_argument("--head-dims", default=None, metavar="DK,DV",
+                    help="override the prefill head sizes (64 or 128 each; timing other shapes), not the headline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-states", action="store_true", help="skip the state-emission (every 512 tokens) timing")
     ap.add_argument("--no-long", action="store_true", help="skip the long-context (T = 65536) timing")
@@ -571,6 +576,9 @@ def main():
     if args.prefill_shape:
         B, T, H = (int(x) for x in args.prefill_shape.split(","))
         PREFILL.update(B=B, T=T, H=H, name=f"prefill_b{B}_t{T}_h{H}")
+    if args.head_dims:
+        dk, dv = (int(x) for x in args.head_dims.split(","))
+        PREFILL.update(dk=dk, dv=dv, name=f"{PREFILL['name']}_dk{dk}_dv{dv}")
     if args.decode_batch:
         DECODE.update(batch=args.decode_batch, name=f"decode_b{args.decode_batch}_h{DECODE['H']}")
     if args.impl == "reference":

@@ -70,11 +70,12 @@ typedef enum { KDA_DTYPE_BF16 = 0, KDA_DTYPE_FP32 = 1 } kda_dtype;
 
 /* Prefill kernel selection for kda_forward_chunked_impl. */
 typedef enum {
-    KDA_IMPL_AUTO = 0,    /* bf16 inputs: the tcgen05 kernel (dk = dv = 128; any other bf16 head size
-                             is refused with KDA_ERR_UNSUPPORTED, never run token-serially without
-                             being asked); fp32 inputs: the SIMT kernel (the only fp32 kernel: bf16
-                             tensor-core operands cannot meet an fp32 accuracy bar) */
-    KDA_IMPL_TCGEN05 = 1, /* chunkwise tensor-core kernel: bf16, dk = dv = 128 only */
+    KDA_IMPL_AUTO = 0,    /* bf16 inputs: the tcgen05 kernel (every supported head size); fp32
+                             inputs: the SIMT kernel (the only fp32 kernel: bf16 tensor-core
+                             operands cannot meet an fp32 accuracy bar) */
+    KDA_IMPL_TCGEN05 = 1, /* chunkwise tensor-core kernel: bf16, dk and dv each 64 or 128.  It
+                             always computes 128 x 128 states; a head size of 64 is embedded in
+                             them with zero channels (exact), so it costs what 128 does */
     KDA_IMPL_SIMT = 2     /* token-serial fp32 CUDA-core kernel: every supported dtype and size */
 } kda_impl;
 
@@ -94,9 +95,8 @@ typedef enum {
  *             between outputs and inputs is not allowed.
  *   dtype   : kda_dtype.
  *
- * Kernel: KDA_IMPL_AUTO (see kda_impl): bf16 with dk = dv = 128 runs the chunkwise tensor-core
- * kernel, fp32 the fp32 kernel; bf16 with another head size returns KDA_ERR_UNSUPPORTED (use
- * kda_forward_chunked_impl with KDA_IMPL_SIMT for it).
+ * Kernel: KDA_IMPL_AUTO (see kda_impl): bf16 runs the chunkwise tensor-core kernel, fp32 the
+ * fp32 kernel.
  *
  * Returns KDA_OK, or a negative kda_status (nothing is enqueued on error).
  */

@@ -141,9 +141,9 @@ int forward_impl(const void* q, const void* k, const void* v, const void* g, con
                        interval, n_mid, cu_seqlens, fused};
     const bool tc_ok = kda::prefill_tc_supports(a);
     if (impl == KDA_IMPL_TCGEN05 && !tc_ok) return KDA_ERR_UNSUPPORTED;
-    // AUTO: the chunkwise tensor-core kernel for bf16 (dk = dv = 128), the fp32 kernel for fp32
-    // inputs; a bf16 shape the tensor-core kernel does not cover is refused rather than sent to the
-    // token-serial kernel behind the caller's back (KDA_IMPL_SIMT runs it when asked for)
+    // AUTO: the chunkwise tensor-core kernel for bf16 (every supported head size), the fp32 kernel
+    // for fp32 inputs; a bf16 shape the tensor-core kernel did not cover would be refused rather than
+    // sent to the token-serial kernel behind the caller's back (KDA_IMPL_SIMT runs it when asked for)
     if (impl == KDA_IMPL_AUTO && dtype == KDA_DTYPE_BF16 && !tc_ok) return KDA_ERR_UNSUPPORTED;
     if (T == 0) {
         // No tokens: the final state is the initial state.

@@ -96,7 +96,7 @@ int validate(const void* q, const void* k, const void* v, const void* g, const v
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
     // the kernel choice of kda_forward_chunked_impl, checked here so that a refusal comes before
     // any copy is enqueued
-    const bool tc_shape = dtype == KDA_DTYPE_BF16 && dk == 128 && dv == 128;
+    const bool tc_shape = dtype == KDA_DTYPE_BF16;   // head sizes 64 and 128 both (checked above)
     if (impl == KDA_IMPL_TCGEN05 && !tc_shape) return KDA_ERR_UNSUPPORTED;
     if (impl == KDA_IMPL_AUTO && dtype == KDA_DTYPE_BF16 && !tc_shape) return KDA_ERR_UNSUPPORTED;
     if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;

@@ -1,5 +1,6 @@
 // KDA chunked prefill on sm_100a: TMA loads, tcgen05 tensor-core products with TMEM
-// accumulators, fp32 state carried across 64-token chunks.  bf16 inputs, dk = dv = 128.
+// accumulators, fp32 state carried across 64-token chunks.  bf16 inputs; dk and dv each 64 or
+// 128, every product 128 wide (see "Head size 64" below).
 //
 // Method (chunk-recurrent form of the gated delta rule: podcast show-notes section 2.1,
 // RetNet chunk recurrence + Gated DeltaNet gated delta rule; delta rule of the "Day 21"
@@ -39,6 +40,14 @@
 //                      products, another the O store and the v loads.
 // All tcgen05 products are M = 128: products with 64 meaningful rows read 64 further rows
 // of other valid shared memory into TMEM lanes that are never read.
+//
+// Head size 64.  The kernel always works on 128 key channels and 128 value columns.  The tensor
+// maps of q, k, g (and v, o) are declared with the true channel count, so the TMA box of
+// channels 64-127 of a 64-wide tensor lies wholly outside it and lands as zeros.  That is an
+// exact embedding of the smaller problem: a key channel with k = q = 0 and g = 0 (or any bounded
+// decay) leaves its state row at zero and adds nothing to A, P or O; a value column with v = 0
+// leaves its state column, Y, U and O column at zero.  Only the state's row and column strides,
+// and the O store of columns 64-127, depend on dk and dv.
 #include <cudaTypedefs.h>
 #include <mutex>
 
@@ -51,13 +60,14 @@ namespace {
 using namespace sm100;
 
 constexpr int kC = 64;          // chunk length
-constexpr int kD = 128;         // dk = dv
+constexpr int kD = 128;         // key channels and value columns the kernel works on (dk, dv <= kD)
 constexpr int kThreads = 512;   // 16 warps
 constexpr int kPrepThreads = 256;
 constexpr int kSerialThreads = 256;
 constexpr uint32_t kBarPrep = 1, kBarSerial = 2;   // named hardware barriers
 constexpr int kIssuer = 0;                         // prep thread that issues the g loads (and chunk 0's q, k) and signals
 constexpr int kMma1Issuer = 224;                   // prep thread that issues MMA1 (warp 7: lightest in the solve)
+constexpr int kGateWarp0 = 10, kGateWarps = 6;     // with the prologue: the recurrence warps that convert the gate
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
 constexpr uint32_t OFF_RAW_Q = 0;           // TMA destination, bf16 [64 tok][128], 2 boxes of 8 KB
@@ -110,6 +120,7 @@ struct TcParams {
     int interval, n_mid;
     const int* cu_seqlens;          // packed sequences (B sequences over T tokens), or null
     int B, T, H;
+    int dk, dv;                     // 64 or 128 each: the state's row / column counts in memory
 };
 
 // Element-wise bf16x2 product, rounded to nearest even.
@@ -198,8 +209,23 @@ __device__ __forceinline__ float ex2_approx(float x);
 // sigmoid with lower bound -5 of the skill card's quick facts).  1 + e^{-z} overflows to inf for
 // z << 0, which gives 0 (no decay / no write), the limit.
 __device__ __forceinline__ float sigmoid_fast(float z) { return __fdividef(1.f, 1.f + ex2_approx(-z * 1.4426950408889634f)); }
-__device__ __forceinline__ float log_decay_from_logit(float z) {
-    return __fdividef(-5.f, 1.f + ex2_approx(-z * 1.4426950408889634f));
+// The log-decay g = -5 sigmoid(z) of a pair of logits, scaled by 2^11 and rounded to an f16 pair.
+// The prologue converts each chunk's gate logits in place to this form ahead of the scan.  The
+// relative error is at most 2^-11; the scale keeps every |g| >= 2^-25 a normal f16 (below that the
+// absolute error is under 2^-36), and 5 * 2^11 stays under the f16 maximum.
+__device__ __forceinline__ uint32_t gate_f16x2_from_logits(uint32_t zz) {
+    const float z0 = __uint_as_float(zz << 16), z1 = __uint_as_float(zz & 0xFFFF0000u);
+    const float g0 = __fdividef(-5.f * 2048.f, 1.f + ex2_approx(-z0 * 1.4426950408889634f));
+    const float g1 = __fdividef(-5.f * 2048.f, 1.f + ex2_approx(-z1 * 1.4426950408889634f));
+    uint32_t h;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(g1), "f"(g0));
+    return h;
+}
+__device__ __forceinline__ float2 f32x2_from_f16x2(uint32_t h) {
+    float lo, hi;
+    asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+        : "=f"(lo), "=f"(hi) : "r"(h));
+    return make_float2(lo, hi);
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -251,10 +277,11 @@ __device__ __forceinline__ void ldsm_b16x8_trans(uint32_t base, uint32_t row_byt
 // formed first), X_RJ = -sum_{L=J}^{R-1} At_RL X_LJ for R = J+1 .. 3, so the dependent chain is one
 // accumulation per block.  Each X_LJ it needs is the diagonal block (level 0's transposed copy) or
 // one it has just formed, kept as a B fragment in registers: no other warp is waited for.  T =
-// X Diag(beta) entries are written as they are formed.  (bf16 operands at these points leave the
-// output error unchanged in the chunk model.)
+// X Diag(beta) entries are written as they are formed, row r times rowf[r] when rowf is given.
+// (bf16 operands at these points leave the output error unchanged in the chunk model.)
 template <int J>
-__device__ __forceinline__ void offdiag_column(uint32_t sb, const float* beta, uint8_t* sm, int nt, int lane) {
+__device__ __forceinline__ void offdiag_column(uint32_t sb, const float* beta, const float* rowf, uint8_t* sm, int nt,
+                                               int lane) {
     constexpr int NR = 3 - J;   // blocks below the diagonal in this column
     const int g4 = lane >> 2, t4 = lane & 3;
     uint32_t at[NR][NR][4];     // A fragments of At_RL, [R - J - 1][L - J]
@@ -284,10 +311,15 @@ __device__ __forceinline__ void offdiag_column(uint32_t sb, const float* beta, u
         float x[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int L = J; L < R; ++L) mma_16816(x, at[R - J - 1][L - J], xb[L - J]);
-        *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(16 * R + g4), col, 8192)) =
-            pack_bf16x2(mul2(make_float2(-x[0], -x[1]), make_float2(b0, b1)));
-        *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(16 * R + g4 + 8), col, 8192)) =
-            pack_bf16x2(mul2(make_float2(-x[2], -x[3]), make_float2(b0, b1)));
+        float2 t0v = mul2(make_float2(-x[0], -x[1]), make_float2(b0, b1));
+        float2 t1v = mul2(make_float2(-x[2], -x[3]), make_float2(b0, b1));
+        if (rowf) {
+            const float f0 = rowf[16 * R + g4], f1 = rowf[16 * R + g4 + 8];
+            t0v = mul2(t0v, make_float2(f0, f0));
+            t1v = mul2(t1v, make_float2(f1, f1));
+        }
+        *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(16 * R + g4), col, 8192)) = pack_bf16x2(t0v);
+        *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(16 * R + g4 + 8), col, 8192)) = pack_bf16x2(t1v);
         if (R < 3) {
             xb[R - J][0] = movmatrix_trans(pack_bf16x2(-x[0], -x[1]));
             xb[R - J][1] = movmatrix_trans(pack_bf16x2(-x[2], -x[3]));
@@ -295,8 +327,12 @@ __device__ __forceinline__ void offdiag_column(uint32_t sb, const float* beta, u
     }
 }
 
-// kFused: the gate and normalisation prologue (q, k raw; g, beta as logits).  kPacked: packed
-// variable-length sequences.  Compiled separately so that the plain path carries neither.
+// kFused: the gate and normalisation prologue (q, k raw; g, beta as logits).  Its extra work is kept
+// off the prep group's path where it can be: six recurrence warps convert the gate logits to log-decays
+// two chunks ahead, while they would otherwise wait for the next MMA3; the operand tiles are those of
+// the raw q, k, and the row norms (one pass after the tiles) are applied where elements are scaled
+// anyway.  kPacked: packed variable-length sequences.  Compiled separately so that the plain path
+// carries neither.
 template <bool kFused, bool kPacked>
 __global__ void __launch_bounds__(kThreads, 1)
 kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -312,12 +348,13 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // TMA / MMA completion barriers (one phase per chunk) and prep -> serial hand-offs.
     __shared__ uint64_t bar_qk, bar_g, bar_v, bar_ap, bar_c, bar_u, bar_os, bar_kq, bar_tpk;
     __shared__ uint64_t bar_drain_p, bar_drain_s, bar_drain_g;
+    __shared__ uint64_t bar_gc;   // with the prologue: a chunk's gate converted (one arrival per converting warp)
     __shared__ uint32_t tmem_base_s;
     __shared__ __align__(16) float s_beta[kC];
     __shared__ __align__(16) float s_gamma[2][kD];     // e^{Gam_63} per channel, by chunk parity (float2 stores)
     __shared__ __align__(16) float s_qsum[4][kD];      // g summed over each 16-token quarter
     __shared__ __align__(16) float s_g1648[2][kD];     // g of tokens 16 and 48 (raw g is dead after the scan)
-    __shared__ float s_norm[2 * kC];                   // with the prologue: 1/|q_t|, then 1/|k_t|
+    __shared__ __align__(16) float s_norm[2][2 * kC];  // with the prologue: 1/|q_t|, then 1/|k_t|, by chunk parity
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     auto tid_is_zero = [&]() { return tid == 0; };
@@ -345,6 +382,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         mbar_init(&bar_qk, 1); mbar_init(&bar_g, 1); mbar_init(&bar_v, 1); mbar_init(&bar_ap, 1);
         mbar_init(&bar_c, 1); mbar_init(&bar_u, 1); mbar_init(&bar_os, 1); mbar_init(&bar_kq, 1);
         mbar_init(&bar_tpk, 1); mbar_init(&bar_drain_p, 1); mbar_init(&bar_drain_s, 1); mbar_init(&bar_drain_g, 1);
+        mbar_init(&bar_gc, kGateWarps);
         fence_mbar_init();
         prefetch_tensormap(&tm_q); prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_g); prefetch_tensormap(&tm_v); prefetch_tensormap(&tm_o);
@@ -414,7 +452,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 s_beta[ptid] = kFused ? (chunk * kC + ptid < T ? sigmoid_fast(bz) : 0.f) : bz;
             }
             if (chunk + 1 < nchunks) beta_next = fetch_beta(chunk + 1);
-            ok = mbar_wait(&bar_g, par, p.timeout_ns);     // every thread: its own view of the TMA data
+            // every thread: its own view of the TMA data (with the prologue: of the converted gate,
+            // which recurrence warps write into the MMA1 A space from the TMA data)
+            ok = mbar_wait(kFused ? &bar_gc : &bar_g, par, p.timeout_ns);
             if (ok && ptid == kIssuer) pending_g = -1;
             // ---- P2: Gam = in-chunk prefix sum of g in fp32: the running sum over this quarter,
             // then the totals of the quarters before it
@@ -426,9 +466,17 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const uint32_t w = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_G + sw128_offset(16 * tq + i, ch0, 8192));
-                    float g0 = __uint_as_float(w << 16), g1 = __uint_as_float(w & 0xFFFF0000u);
-                    if (kFused) { g0 = log_decay_from_logit(g0); g1 = log_decay_from_logit(g1); }
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(sm + (kFused ? OFF_A1 : OFF_RAW_G) +
+                                                                          sw128_offset(16 * tq + i, ch0, 8192));
+                    float g0, g1;
+                    if (kFused) {   // 2^11 g in f16 (exact rescaling)
+                        const float2 h = f32x2_from_f16x2(w);
+                        g0 = h.x * 0x1p-11f;
+                        g1 = h.y * 0x1p-11f;
+                    } else {
+                        g0 = __uint_as_float(w << 16);
+                        g1 = __uint_as_float(w & 0xFFFF0000u);
+                    }
                     if ((kFused || kPacked) && 16 * tq + i >= nvalid) g0 = g1 = 0.f;
                     acc = add2(acc, make_float2(g0, g1));
                     gam[i] = acc;
@@ -440,30 +488,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             ok = named_bar_and(kBarPrep, kPrepThreads, ok);
             if (!ok) break;
             // raw g of this chunk is consumed: load the next chunk's
-            if (ptid == kIssuer && chunk + 1 < nchunks) { load_g(chunk + 1); pending_g = chunk + 1; }
-            if (kFused) {   // the norms below read raw q and k
-                ok = mbar_wait(&bar_qk, par, p.timeout_ns);
-                if (ok && ptid == kIssuer) pending_qk = -1;
-            }
-            if (kFused) {
-                // 1/|x| of every q and k row of the chunk (row = thread/2, 64 channels per thread)
-                const int row = ptid >> 1, half = ptid & 1, t = row & (kC - 1);
-                const uint8_t* tile = sm + (row < kC ? OFF_RAW_Q : OFF_RAW_K) + half * 8192 + t * 128;
-                float2 ss2 = make_float2(0.f, 0.f);   // even and odd channels
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint4 w4 = *reinterpret_cast<const uint4*>(tile + ((j ^ (t & 7)) << 4));
-                    const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 x2 = make_float2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
-                        ss2 = fma2(x2, x2, ss2);
-                    }
-                }
-                float ss = ss2.x + ss2.y;
-                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                if (half == 0) s_norm[row] = ss > 0.f ? rsqrtf(ss) : 0.f;
-            }
+            // (with the prologue the recurrence warps that convert the gate load it)
+            if (!kFused && ptid == kIssuer && chunk + 1 < nchunks) { load_g(chunk + 1); pending_g = chunk + 1; }
             {
                 float2 carry = make_float2(0.f, 0.f);
 #pragma unroll 1
@@ -493,15 +519,11 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     make_float2(ex2_approx_sub(r63[0] * kLog2e), ex2_approx_sub(r63[1] * kLog2e));
             // ---- P3: operand tiles (KQ may be rewritten once MMA3 of the previous chunk is done;
             // every thread waits for that itself, the vote is at the next barrier)
-            if (!kFused && ok) {
+            if (ok) {
                 ok = mbar_wait(&bar_qk, par, p.timeout_ns);
                 if (ok && ptid == kIssuer) pending_qk = -1;
             }
             if (chunk > 0 && ok) ok = mbar_wait(&bar_c, ppar, p.timeout_ns);
-            if (kFused) {   // the inverse norms are read below
-                ok = named_bar_and(kBarPrep, kPrepThreads, ok);
-                if (!ok) break;
-            }
             uint32_t kb[16];  // Kb of these tokens, written once the previous chunk released the tile
             {
                 // per channel, against the block's reference token m: Gam_m*log2e, e^{Gam_63-Gam_m},
@@ -540,30 +562,18 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     uint32_t qw = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_Q + sw128_offset(t, ch0, 8192));
                     uint32_t kw = *reinterpret_cast<const uint32_t*>(sm + OFF_RAW_K + sw128_offset(t, ch0, 8192));
                     if (kPacked && t >= nvalid) qw = kw = 0u;
-                    float2 qv = make_float2(__uint_as_float(qw << 16), __uint_as_float(qw & 0xFFFF0000u));
-                    float2 kv = make_float2(__uint_as_float(kw << 16), __uint_as_float(kw & 0xFFFF0000u));
-                    if (kFused) {
-                        const float qn = s_norm[t], kn = s_norm[kC + t];
-                        qv = mul2(qv, make_float2(qn, qn));
-                        kv = mul2(kv, make_float2(kn, kn));
-                    }
+                    const float2 kv = make_float2(__uint_as_float(kw << 16), __uint_as_float(kw & 0xFFFF0000u));
                     const float2 x = fma2(gam[i], make_float2(kLog2e, kLog2e), ngmL);
                     const float2 E = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                     const float2 I = make_float2(ex2_approx(-x.x), ex2_approx(-x.y));
                     const float2 kI = mul2(kv, I);
-                    // MMA1 operands: A rows [Qt0;Kt0;Qt1;Kt1], B rows [Kh0(16);Kh1(48);Kh0(48)].  Without
-                    // the prologue q and k are bf16 already: bf16 q (k) times the bf16-rounded factor
-                    uint32_t a1q, a1k, b1;
-                    if (kFused) {
-                        a1q = pack_bf16x2(mul2(qv, E));
-                        a1k = pack_bf16x2(mul2(kv, E));
-                        b1 = pack_bf16x2(kI);
-                    } else {
-                        const uint32_t e2 = pack_bf16x2(E), i2 = pack_bf16x2(I);
-                        a1q = mul_bf16x2(qw, e2);
-                        a1k = mul_bf16x2(kw, e2);
-                        b1 = mul_bf16x2(kw, i2);
-                    }
+                    // MMA1 operands: A rows [Qt0;Kt0;Qt1;Kt1], B rows [Kh0(16);Kh1(48);Kh0(48)]: bf16 q (k)
+                    // times the bf16-rounded factor.  With the prologue q and k are the raw rows here;
+                    // their norms are applied further on (see the norm pass below)
+                    const uint32_t e2 = pack_bf16x2(E), i2 = pack_bf16x2(I);
+                    const uint32_t a1q = mul_bf16x2(qw, e2);
+                    const uint32_t a1k = mul_bf16x2(kw, e2);
+                    const uint32_t b1 = mul_bf16x2(kw, i2);
                     *reinterpret_cast<uint32_t*>(sm + OFF_A1 + sw128_offset(rq, ch0, 16384)) = a1q;
                     *reinterpret_cast<uint32_t*>(sm + OFF_A1 + sw128_offset(rk, ch0, 16384)) = a1k;
                     *reinterpret_cast<uint32_t*>(sm + OFF_BB + sw128_offset(t, ch0, 12288)) = b1;
@@ -578,6 +588,31 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     *reinterpret_cast<uint32_t*>(sm + OFF_KQ + sw128_offset(rk, ch0, 16384)) = mul_bf16x2(a1k, cmb);
                     kb[i] = pack_bf16x2(mul2(kI, ce));
                 }
+            }
+            if (kFused) {
+                // 1/|x| of every raw q and k row of the chunk (row = thread/2, 64 channels per thread).
+                // q and k enter every product of the chunk linearly, so their norms are applied where
+                // an element is scaled anyway, not to the operand tiles: 1/|k| on A (row and column),
+                // on the rows of T and on Kt S in Y; 1/|q| on O.  (With Kn = Diag(1/|k|): A' = Diag(beta)
+                // Kn A Kn, U' = T' (V - Kn Kt S); MMA5 and MMA6 then take U~ = Kn U' with the raw P and Kb,
+                // since P' = Diag(1/|q|) P Kn and Kb' = Kn Kb.)  This pass runs after the operand tiles,
+                // off their path, and before the hand-off that lets the next q, k overwrite the raw tiles.
+                const int row = ptid >> 1, half = ptid & 1, t = row & (kC - 1);
+                const uint8_t* tile = sm + (row < kC ? OFF_RAW_Q : OFF_RAW_K) + half * 8192 + t * 128;
+                float2 ss2 = make_float2(0.f, 0.f);   // even and odd channels
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint4 w4 = *reinterpret_cast<const uint4*>(tile + ((j ^ (t & 7)) << 4));
+                    const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 x2 = make_float2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
+                        ss2 = fma2(x2, x2, ss2);
+                    }
+                }
+                float ss = ss2.x + ss2.y;
+                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                if (half == 0) s_norm[par][row] = ss > 0.f ? rsqrtf(ss) : 0.f;
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
@@ -638,11 +673,12 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     // A row r: strictly lower, scaled by beta_r (select first: masked entries may be inf),
                     // in bf16; the diagonal block's 16 entries also in fp32 (quarter 1 with columns
                     // 0-31 and quarter 3 with columns 32-63 hold the diagonal blocks)
-                    const float br = s_beta[r];
+                    const float br = kFused ? s_beta[r] * s_norm[par][kC + r] : s_beta[r];
                     float w[32];
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
-                        const float2 pr = mul2(make_float2(row[j], row[j + 1]), make_float2(br, br));
+                        float2 pr = mul2(make_float2(row[j], row[j + 1]), make_float2(br, br));
+                        if (kFused) pr = mul2(pr, *reinterpret_cast<const float2*>(&s_norm[par][kC + jb + j]));
                         w[j] = (jb + j < r) ? pr.x : 0.f;
                         w[j + 1] = (jb + j + 1 < r) ? pr.y : 0.f;
                     }
@@ -702,8 +738,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         const int row = g4 + 8 * hr;
                         const float x0 = xm[nt][2 * hr], x1 = xm[nt][2 * hr + 1];
                         *reinterpret_cast<uint32_t*>(sm + OFF_XD + ((o0 + row) * kLdX + col) * 2) = pack_bf16x2(x0, x1);
-                        *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(o0 + row), o0 + col, 8192)) =
-                            pack_bf16x2(mul2(make_float2(x0, x1), make_float2(b0, b1)));
+                        float2 tv = mul2(make_float2(x0, x1), make_float2(b0, b1));
+                        if (kFused) { const float f = s_norm[par][kC + o0 + row]; tv = mul2(tv, make_float2(f, f)); }
+                        *reinterpret_cast<uint32_t*>(sm + OFF_T + sw128_offset(tp_row(o0 + row), o0 + col, 8192)) = pack_bf16x2(tv);
                     }
                 }
             }
@@ -711,9 +748,10 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             // off-diagonal blocks, one block column per warp pair (8 output columns per warp)
             if (warp < 6) {
                 const int nt = warp & 1;
-                if (warp < 2) offdiag_column<0>(sb, s_beta, sm, nt, lane);
-                else if (warp < 4) offdiag_column<1>(sb, s_beta, sm, nt, lane);
-                else offdiag_column<2>(sb, s_beta, sm, nt, lane);
+                const float* rowf = kFused ? &s_norm[par][kC] : nullptr;
+                if (warp < 2) offdiag_column<0>(sb, s_beta, rowf, sm, nt, lane);
+                else if (warp < 4) offdiag_column<1>(sb, s_beta, rowf, sm, nt, lane);
+                else offdiag_column<2>(sb, s_beta, rowf, sm, nt, lane);
             }
             fence_proxy_async_smem();
             named_bar_sync(kBarPrep, kPrepThreads);
@@ -738,6 +776,41 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // the I/O thread (stid 32) stores O and loads the next v, so that the wait for the O store to
         // have read its staging tile never holds up the next chunk's MMA3.
         int pending = -1;                                   // I/O thread: chunk whose v load is in flight
+        // With the prologue warps kGateWarp0.. of this group convert each chunk's gate logits (bf16 z ->
+        // f16 2^11 g), two chunks ahead of the prep group's scan, in the time they otherwise wait for the
+        // next chunk's MMA3.  The result goes to the MMA1 A space, free from the completion of the
+        // previous chunk's MMA1 (which also means the scan and operand tiles before it are done) to
+        // the next scan; the raw g buffer is then free at once and the next chunk's g is loaded.  No
+        // wait here can see a phase ahead: the next g load, MMA1 and conversion all follow this one.
+        int pending_g = -1;                                 // gate loader (warp kGateWarp0, lane 0)
+        const bool gate_warp = kFused && warp >= kGateWarp0 && warp < kGateWarp0 + kGateWarps;
+        auto convert_gate = [&](int c) -> bool {
+            bool got = c == 0 || mbar_wait(&bar_ap, (uint32_t)((c - 1) & 1), p.timeout_ns);
+            got = got && mbar_wait(&bar_g, (uint32_t)(c & 1), p.timeout_ns);
+            if (got) {
+                const uint4* src = reinterpret_cast<const uint4*>(sm + OFF_RAW_G);
+                uint4* dst = reinterpret_cast<uint4*>(sm + OFF_A1);
+#pragma unroll 1
+                for (int idx = tid - 32 * kGateWarp0; idx < kC * kD * 2 / 16; idx += 32 * kGateWarps) {
+                    const uint4 w = src[idx];
+                    dst[idx] = make_uint4(gate_f16x2_from_logits(w.x), gate_f16x2_from_logits(w.y),
+                                          gate_f16x2_from_logits(w.z), gate_f16x2_from_logits(w.w));
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_gc);
+            if (warp == kGateWarp0 && lane == 0) {
+                // every converting warp has read the raw tile: the next chunk's g may land on it
+                got = mbar_wait(&bar_gc, (uint32_t)(c & 1), p.timeout_ns) && got;
+                if (pending_g == c) pending_g = -1;
+                if (got && c + 1 < nchunks) {
+                    fence_proxy_async_smem();
+                    load_g(c + 1);
+                    pending_g = c + 1;
+                }
+            }
+            return got;
+        };
         int pending_qk = -1;                                // leader: last chunk whose q,k loads it issued
         // Once the prep group has published chunk c's operand tiles (bar_kq): MMA3 = [Qt0;Kt0;Qt1;Kt1] S
         // and the raw q, k of chunk c+1 into the buffers the prep group has finished reading.
@@ -752,8 +825,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const int i = 32 * quarter + lane;
             const int cb0 = 64 * colhalf;
             float r[64];
-            if (p.S0) {
-                const float4* src = reinterpret_cast<const float4*>(p.S0 + ((size_t)bh * kD + i) * kD + cb0);
+            if (p.S0 && i < p.dk && cb0 < p.dv) {
+                const float4* src = reinterpret_cast<const float4*>(p.S0 + ((size_t)bh * p.dk + i) * p.dv + cb0);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const float4 x = src[j];
@@ -780,6 +853,15 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             ok = mbar_wait(&bar_kq, 0u, p.timeout_ns);
             if (ok) issue_for_chunk(0);
         }
+        if (gate_warp) {   // the gates of chunks 0 and 1 (the loop converts chunk c + 2)
+            if (warp == kGateWarp0 && lane == 0 && nchunks > 0) pending_g = 0;   // loaded by the prep group
+            if (nchunks > 0 && !convert_gate(0)) ok = false;
+            if (nchunks > 1 && !convert_gate(1)) ok = false;
+        }
+        // With the prologue every thread of this group reads the chunk's norms, which the prep group
+        // writes before the KQ hand-off: each waits for that hand-off itself.  (The next phase of
+        // bar_kq needs this chunk's MMA3 to have completed, so the parity cannot be a phase ahead.)
+        if (kFused && stid != 0 && nchunks > 0 && ok) ok = mbar_wait(&bar_kq, 0u, p.timeout_ns);
         for (int chunk = 0; chunk < nchunks; ++chunk) {
             const uint32_t par = chunk & 1;
             const int t0 = chunk * kC;
@@ -794,6 +876,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const int tj = 32 * (quarter >> 1) + lane;
                 float ks[64];
                 tmem_ld64(tlane + TM_C + 64 * colhalf, ks);
+                // with the prologue Kt S is that of the raw k row: Y = V - (Kt S) / |k|
+                const float nk = kFused ? -s_norm[par][kC + tj] : -1.f;
 #pragma unroll
                 for (int j = 0; j < 64; j += 8) {
                     const uint32_t off = sw128_offset(tj, 64 * colhalf + j, 8192);
@@ -802,7 +886,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     float y[8];
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
-                        const float2 yy = sub2(__bfloat1622float2(v2[m]), make_float2(ks[j + 2 * m], ks[j + 2 * m + 1]));
+                        const float2 yy = kFused ? fma2(make_float2(ks[j + 2 * m], ks[j + 2 * m + 1]), make_float2(nk, nk),
+                                                        __bfloat1622float2(v2[m]))
+                                                 : sub2(__bfloat1622float2(v2[m]), make_float2(ks[j + 2 * m], ks[j + 2 * m + 1]));
                         y[2 * m] = yy.x;
                         y[2 * m + 1] = yy.y;
                     }
@@ -875,8 +961,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int j = 0; j < 64; j += 8)
                     *reinterpret_cast<uint4*>(sm + OFF_SB + sw128_offset(i, 64 * colhalf + j, 16384)) = pack8(sv + j);
                 // the state after a multiple of the interval (only a full chunk can end on one)
-                if (p.n_mid > 0 && t0 + kC <= T && (t0 + kC) % p.interval == 0) {
-                    float* dst = p.S_mid + (((size_t)bh * p.n_mid + (t0 + kC) / p.interval - 1) * kD + i) * kD + 64 * colhalf;
+                if (p.n_mid > 0 && t0 + kC <= T && (t0 + kC) % p.interval == 0 && i < p.dk && 64 * colhalf < p.dv) {
+                    float* dst = p.S_mid + (((size_t)bh * p.n_mid + (t0 + kC) / p.interval - 1) * p.dk + i) * p.dv + 64 * colhalf;
 #pragma unroll
                     for (int j = 0; j < 64; j += 4)
                         __stcs(reinterpret_cast<float4*>(dst + j), make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]));
@@ -889,9 +975,18 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const int r = 32 * (quarter >> 1) + lane;   // token row of the chunk
                 float ov[64];
                 tmem_ld64(tlane + TM_C + 64 * colhalf, ov);   // warp-collective
+                if (kFused) {   // O of the raw q row: O' = O / |q|
+                    const float nq = s_norm[par][r];
+#pragma unroll
+                    for (int j = 0; j < 64; j += 2) {
+                        const float2 x = mul2(make_float2(ov[j], ov[j + 1]), make_float2(nq, nq));
+                        ov[j] = x.x;
+                        ov[j + 1] = x.y;
+                    }
+                }
                 if (row_stores) {
-                    if (t0 + r < T) {
-                        uint4* orow = reinterpret_cast<uint4*>(p.o + ((row0 + t0 + r) * p.H + h) * kD + 64 * colhalf);
+                    if (t0 + r < T && 64 * colhalf < p.dv) {
+                        uint4* orow = reinterpret_cast<uint4*>(p.o + ((row0 + t0 + r) * p.H + h) * p.dv + 64 * colhalf);
 #pragma unroll
                         for (int j = 0; j < 8; ++j) orow[j] = pack8(ov + 8 * j);
                     }
@@ -908,7 +1003,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 // rows past the tensor's T are clipped by the tensor map
                 if (!row_stores) {
                     tma_store_4d(&tm_o, sm + OFF_V, 0, h, tok0 + t0, bmap);
-                    tma_store_4d(&tm_o, sm + OFF_V + 8192, 64, h, tok0 + t0, bmap);
+                    if (p.dv > 64) tma_store_4d(&tm_o, sm + OFF_V + 8192, 64, h, tok0 + t0, bmap);
                     bulk_commit_group();
                 }
                 if (chunk + 1 < nchunks) {
@@ -921,12 +1016,15 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 ok = mbar_wait(&bar_kq, par ^ 1u, p.timeout_ns);
                 if (ok) issue_for_chunk(chunk + 1);
             }
+            if (kFused && stid != 0 && chunk + 1 < nchunks && ok) ok = mbar_wait(&bar_kq, par ^ 1u, p.timeout_ns);
+            if (gate_warp && chunk + 2 < nchunks && !convert_gate(chunk + 2)) ok = false;
         }
         if (!ok && stid == 0) report_status(p.status, KDA_ERR_TIMEOUT);
         if (stid == 32) {
             bulk_wait_all();
             if (pending >= 0) (void)mbar_wait(&bar_v, (uint32_t)(pending & 1), p.timeout_ns);
         }
+        if (pending_g >= 0) (void)mbar_wait(&bar_g, (uint32_t)(pending_g & 1), p.timeout_ns);
         if (stid == 0) {
             mma_commit(&bar_drain_s);
             if (!mbar_wait(&bar_drain_s, 0, p.timeout_ns)) report_status(p.status, KDA_ERR_TIMEOUT);
@@ -936,11 +1034,14 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tc_fence_after_sync();
         if (ok && p.ST) {
             const int i = 32 * quarter + lane;
-            float* dst = p.ST + ((size_t)bh * kD + i) * kD + 64 * colhalf;
             float sv[64];
-            tmem_ld64(tlane + TM_S + 64 * colhalf, sv);
+            tmem_ld64(tlane + TM_S + 64 * colhalf, sv);   // warp-collective
+            if (i < p.dk && 64 * colhalf < p.dv) {
+                float* dst = p.ST + ((size_t)bh * p.dk + i) * p.dv + 64 * colhalf;
 #pragma unroll
-            for (int j = 0; j < 64; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+                for (int j = 0; j < 64; j += 4)
+                    *reinterpret_cast<float4*>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+            }
         }
     }
     tc_fence_before_sync();
@@ -955,13 +1056,14 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
 }
 
-// [B, T, H, 128] bf16 viewed as a 4-D tensor (d, H, T, B); box = 64 channels x 1 head x 64 tokens.
-// Rows past T read as zeros, which makes the tail of the last chunk an exact no-op.
-bool make_map(CUtensorMap* m, const void* ptr, int B, int T, int H) {
+// [B, T, H, d] bf16 (d = 64 or 128) viewed as a 4-D tensor (d, H, T, B); box = 64 channels x 1 head
+// x 64 tokens.  Rows past T read as zeros, which makes the tail of the last chunk an exact no-op, and
+// so do channels past d (the box at channel 64 of a 64-wide tensor).
+bool make_map(CUtensorMap* m, const void* ptr, int B, int T, int H, int d) {
     auto enc = get_encode_fn();
     if (!enc) return false;
-    cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)T * H * kD * 2};
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
     cuuint32_t box[4] = {64, 1, (cuuint32_t)kC, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
@@ -986,7 +1088,7 @@ void* tensor_map_encoder() {
 }
 
 bool prefill_tc_supports(const PrefillArgs& a) {
-    return a.dtype == KDA_DTYPE_BF16 && a.dk == kD && a.dv == kD;
+    return a.dtype == KDA_DTYPE_BF16 && (a.dk == 64 || a.dk == kD) && (a.dv == 64 || a.dv == kD);
 }
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
@@ -1009,13 +1111,13 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     CUtensorMap mq, mk, mg, mv, mo;
     // packed sequences: one batch entry holding all T tokens
     const int mb = a.cu_seqlens ? 1 : a.B;
-    if (!make_map(&mq, a.q, mb, a.T, a.H) || !make_map(&mk, a.k, mb, a.T, a.H) ||
-        !make_map(&mg, a.g, mb, a.T, a.H) || !make_map(&mv, a.v, mb, a.T, a.H) ||
-        !make_map(&mo, a.o, mb, a.T, a.H))
+    if (!make_map(&mq, a.q, mb, a.T, a.H, a.dk) || !make_map(&mk, a.k, mb, a.T, a.H, a.dk) ||
+        !make_map(&mg, a.g, mb, a.T, a.H, a.dk) || !make_map(&mv, a.v, mb, a.T, a.H, a.dv) ||
+        !make_map(&mo, a.o, mb, a.T, a.H, a.dv))
         return cudaErrorInvalidValue;
     TcParams prm{static_cast<const __nv_bfloat16*>(a.beta), a.S0, static_cast<__nv_bfloat16*>(a.o), a.ST,
                  a.status, a.timeout_ns, a.skip_handoff, a.S_mid, a.interval, a.n_mid, a.cu_seqlens,
-                 a.B, a.T, a.H};
+                 a.B, a.T, a.H, a.dk, a.dv};
     const unsigned grid = (unsigned)((size_t)a.B * a.H);
     if (a.cu_seqlens) {
         if (a.fused) kda_prefill_tc_kernel<true, true><<<grid, kThreads, SMEM_DYN, s>>>(mq, mk, mg, mv, mo, prm);

@@ -110,16 +110,11 @@ def test_forward_rejects_bad_impl(L):
 
 
 def test_forward_tcgen05_rejects_shapes_it_does_not_cover(L):
-    # the tensor-core kernel covers bf16 with dk = dv = 128 only
+    # the tensor-core kernel covers bf16 only (head sizes 64 and 128, like every kernel)
     assert fwd(L, ptrs(), dtype=1, impl=1) == UNSUPPORTED
-    assert fwd(L, ptrs(), dk=64, dv=64, impl=1) == UNSUPPORTED
-
-
-def test_forward_auto_refuses_bf16_shapes_without_a_tensor_core_kernel(L):
-    # AUTO never runs a bf16 problem on the token-serial kernel without being asked
     for dk, dv in ((64, 64), (128, 64), (64, 128)):
-        assert fwd(L, ptrs(), dk=dk, dv=dv, impl=0) == UNSUPPORTED
-        assert fwd(L, ptrs(), dk=dk, dv=dv, impl=0, T=0) == UNSUPPORTED
+        assert fwd(L, ptrs(), dk=dk, dv=dv, dtype=1, impl=1) == UNSUPPORTED
+        assert fwd(L, ptrs(), dk=dk, dv=dv, dtype=1, impl=1, T=0) == UNSUPPORTED
 
 
 def test_decode_rejects_bad_arguments(L):

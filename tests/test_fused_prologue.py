@@ -63,7 +63,7 @@ def gpu_raw(B, T, H, d, dtype, seed, zg_mean=0.0):
     return make_prefill_raw_inputs(B, T, H, d, d, dtype, seed=seed, s0_std=0.05, zg_mean=zg_mean, device="cuda")
 
 
-CASES = [("bf16", "tcgen05", 128, 1, 1000, 4), ("bf16", "simt", 128, 2, 300, 2), ("fp32", "simt", 64, 1, 256, 3),
+CASES = [("bf16", "tcgen05", 128, 1, 1000, 4), ("bf16", "tcgen05", 64, 2, 300, 3), ("bf16", "simt", 128, 2, 300, 2), ("fp32", "simt", 64, 1, 256, 3),
          ("fp32", "simt", 128, 1, 130, 2)]
 
 

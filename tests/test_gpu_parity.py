@@ -97,13 +97,9 @@ def test_prefill_small_fp32_config(impl):
 @pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (128, 64), (64, 128)])
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 200])
 def test_prefill_shapes(impl, dtype, dk, dv, T):
+    # AUTO: bf16 on the tensor-core kernel (head size 64 embedded in its 128-wide tiles), fp32 on
+    # the CUDA-core kernel
     inputs = gpu_inputs(2, T, 3, dk, dv, dtype, s0_std=0.05, seed=T)
-    if impl == "auto" and dtype == "bf16" and (dk, dv) != (128, 128):
-        # AUTO refuses a bf16 head size the tensor-core kernel does not cover
-        with pytest.raises(kda.KdaError) as err:
-            run_prefill(inputs, impl)
-        assert err.value.status == kda.STATUS["KDA_ERR_UNSUPPORTED"]
-        return
     check_prefill(inputs, dtype, impl)
 
 
@@ -173,3 +169,33 @@ def test_prefill_padding_tokens_are_no_ops(impl):
     kp[:, T:] = k[:, :pad]                 # nonzero keys, but beta = 0 and g = 0
     _, ST2 = run_prefill((qp, kp, vp, z(g), z(beta), S0), impl)
     assert torch.equal(ST, ST2) or max_rel_err(to_np(ST2), to_np(ST)) < 1e-6
+
+
+# ---------------------------------------------------------------------- head size 64 on the tensor core
+
+@pytest.mark.parametrize("dk,dv,B,T,H", [(64, 64, 2, 1000, 5), (64, 128, 1, 777, 3), (128, 64, 1, 777, 3)])
+def test_prefill_head64_tensor_core_matches_oracle(dk, dv, B, T, H):
+    """bf16 head size 64 on the chunkwise tensor-core kernel: several chunks and a ragged tail."""
+    check_prefill(gpu_inputs(B, T, H, dk, dv, "bf16", s0_std=0.05, zg_mean=-1.0, seed=31), "bf16", "tcgen05")
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
+def test_prefill_head64_is_the_zero_padded_head128_problem(dk, dv):
+    """The tensor-core kernel computes a head size of 64 as the 128-wide problem with zero channels
+    (q = k = g = 0 past dk, v = 0 past dv).  Running that padded problem explicitly must give the
+    same bits: the outputs' first dv columns, the state's top-left dk x dv block, and zeros elsewhere."""
+    B, T, H = 2, 333, 3
+    q, k, v, g, beta, S0 = gpu_inputs(B, T, H, dk, dv, "bf16", s0_std=0.05, zg_mean=-1.0, seed=32)
+    o, ST = run_prefill((q, k, v, g, beta, S0), "tcgen05")
+
+    def pad(x, d):
+        out = torch.zeros(x.shape[:-1] + (128,), dtype=x.dtype, device=DEV)
+        out[..., :d] = x
+        return out.contiguous()
+
+    S0p = torch.zeros((B, H, 128, 128), dtype=torch.float32, device=DEV)
+    S0p[:, :, :dk, :dv] = S0
+    op, STp = run_prefill((pad(q, dk), pad(k, dk), pad(v, dv), pad(g, dk), beta, S0p), "tcgen05")
+    assert torch.equal(o, op[..., :dv])
+    assert torch.equal(ST, STp[:, :, :dk, :dv])
+    assert not torch.any(op[..., dv:]) and not torch.any(STp[:, :, dk:]) and not torch.any(STp[:, :, :, dv:])

@@ -97,6 +97,7 @@ def _pinned(t):
     (1, 4097, 2, 128, "bf16", "auto", True),        # one token past two segments
     (2, 300, 2, 64, "fp32", "simt", True),          # the CUDA-core kernel
     (2, 4200, 1, 64, "bf16", "simt", False),
+    (2, 4200, 2, 64, "bf16", "tcgen05", True),      # head size 64 on the tensor-core kernel
 ])
 def test_host_prefill_equals_device_prefill_bitwise(B, T, H, d, dtype, impl, s0):
     q, k, v, g, beta, S0 = _inputs(B, T, H, d, dtype, seed=3, s0=s0)

@@ -121,6 +121,8 @@ CASES = [  # (B, T, H, dk, dv, dtype, impl, interval)
     (2, 1100, 3, 128, 128, "bf16", "auto", 512),
     (1, 700, 2, 128, 128, "bf16", "tcgen05", 64),
     (1, 1024, 2, 128, 128, "bf16", "tcgen05", 256),
+    (1, 700, 2, 64, 128, "bf16", "tcgen05", 128),     # head size 64 embedded in the 128-wide tiles
+    (2, 600, 2, 128, 64, "bf16", "tcgen05", 64),
     (2, 300, 2, 64, 128, "fp32", "simt", 64),
     (1, 520, 2, 128, 128, "bf16", "simt", 128),
 ]

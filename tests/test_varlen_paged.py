@@ -99,7 +99,8 @@ def packed_case(lengths, H, d, dtype, seed=0, lead=0, tail=0):
 
 
 @gpu
-@pytest.mark.parametrize("dtype,impl,d", [("bf16", "tcgen05", 128), ("bf16", "simt", 128), ("fp32", "simt", 64)])
+@pytest.mark.parametrize("dtype,impl,d", [("bf16", "tcgen05", 128), ("bf16", "tcgen05", 64), ("bf16", "simt", 128),
+                                          ("fp32", "simt", 64)])
 def test_packed_sequences_match_the_oracle_one_by_one(dtype, impl, d):
     lengths = [1, 63, 64, 65, 200, 0, 130, 7]
     q, k, v, g, beta, cu, S0 = packed_case(lengths, 3, d, dtype, seed=2)

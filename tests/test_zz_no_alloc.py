@@ -74,7 +74,7 @@ def test_bad_arguments_are_refused_before_anything_runs(L):
     assert noalloc(L, fake_ptrs(), T=-1) == INVALID
     assert noalloc(L, fake_ptrs(), impl=9) == INVALID
     assert noalloc(L, fake_ptrs(), dk=96) == UNSUPPORTED
-    assert noalloc(L, fake_ptrs(), dk=64, dv=64, impl=IMPL["auto"]) == UNSUPPORTED    # bf16 off the tensor-core shape
+    assert noalloc(L, fake_ptrs(), dk=64, dv=64, dtype=1, impl=IMPL["tcgen05"]) == UNSUPPORTED   # fp32 has no tensor-core kernel
     assert noalloc(L, fake_ptrs(), dtype=1, impl=IMPL["tcgen05"]) == UNSUPPORTED
     p = fake_ptrs(); p[0] = None
     assert noalloc(L, p) == INVALID
