@@ -101,3 +101,20 @@ def test_zero_query_rows_give_zero_outputs(impl):
     torch.cuda.synchronize()
     assert bool((o[:, 5] == 0).all()) and bool((o[:, 77, 1] == 0).all())
     assert not bool((o[:, 6] == 0).all())
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("d", [128, 64])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 128, 129, 200])
+def test_fused_prefill_chunk_counts(T, d):
+    """The tensor-core kernel's prologue converts the gate of chunks 0 and 1 before its loop and of
+    chunk c + 2 inside it, and loads the next gate after each conversion: one, two and three chunks
+    (and ragged tails) take different paths through that pipeline."""
+    q, k, v, z_g, z_b, S0 = gpu_raw(2, T, 2, d, "bf16", seed=T)
+    o, ST = kda.kda_forward_chunked_fused(q, k, v, z_g, z_b, S0, impl="tcgen05")
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    o_ref, ST_ref = oracle.forward_fused(q, k, v, z_g, z_b, S0)
+    eo = max_rel_err(o.double().cpu().numpy(), o_ref)
+    es = max_rel_err(ST.double().cpu().numpy(), ST_ref)
+    assert eo <= 2e-2 and es <= 2e-2, (eo, es)
