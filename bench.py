@@ -110,6 +110,61 @@ def recorded_traffic(kernel_tag):
     return None
 
 
+def measure_long_split(kda, LC, lq, lo, lst, stream, reps, l_ms):
+    """The long-context workload cut at T/2 the way context parallelism cuts it over ranks, all on one
+    GPU: one launch of 3 x B*H half-length runs (the first halves from S0 = 0; the second halves from
+    a zero state; the second halves with v = 0 and S0 = I, whose outputs are the correction operands
+    and whose final states are the state maps), then the incoming state's composition and the
+    output correction.  Measured to show whether filling the idle SMs this way pays."""
+    import torch
+
+    B, T, H, dk, dv = LC["B"], LC["T"], LC["H"], LC["dk"], LC["dv"]
+    h = T // 2
+    q, k, v, g, beta = lq[:5]
+    cat = lambda x, y, z: torch.cat([x, y, z], 0).contiguous()
+    q3 = cat(q[:, :h], q[:, h:], q[:, h:])
+    k3 = cat(k[:, :h], k[:, h:], k[:, h:])
+    g3 = cat(g[:, :h], g[:, h:], g[:, h:])
+    b3 = cat(beta[:, :h], beta[:, h:], beta[:, h:])
+    v3 = cat(v[:, :h], v[:, h:], torch.zeros_like(v[:, h:]))
+    S03 = torch.zeros((3 * B, H, dk, dv), dtype=torch.float32, device=q.device)
+    S03[2 * B:] = torch.eye(dk, dtype=torch.float32, device=q.device)
+    o3 = torch.empty((3 * B, h, H, dv), dtype=q.dtype, device=q.device)
+    st3 = torch.empty((3 * B, H, dk, dv), dtype=torch.float32, device=q.device)
+    final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+
+    def step(whole):
+        kda.kda_forward_chunked(q3, k3, v3, g3, b3, S03, o=o3, S_T=st3, stream=stream)
+        if whole:   # S_in = N of the first half (it started from 0); o2 += S_in^T C; S_T = M2 S_in + N2
+            kda.kda_output_correct(o3[2 * B:], st3[:B], o3[B:2 * B], out=o3[B:2 * B], stream=stream)
+            kda.kda_state_compose(st3[2 * B:], st3[:B], st3[B:2 * B], out=final, stream=stream)
+
+    times = {}
+    for whole in (False, True):
+        step(whole)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        torch.cuda.synchronize()
+        for e0, e1 in ev:
+            e0.record(stream)
+            step(whole)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        times[whole] = sum(e0.elapsed_time(e1) for e0, e1 in ev) / reps
+    if kda.kda_get_device_status() != 0:
+        raise RuntimeError("device status after the split long-context run")
+    o_split = torch.cat([o3[:B], o3[B:2 * B]], 1).float()
+    ref = lo.float()
+    rel = lambda x, r: float((x - r).abs().max() / r.abs().max())
+    out = {"segments": 2, "ctas": 3 * B * H, "forward_ms": times[False],
+           "correct_and_compose_ms": times[True] - times[False], "total_ms": times[True],
+           "vs_single_pass": times[True] / l_ms,
+           "o_first_half_bitwise_equal": bool(torch.equal(o3[:B], lo[:, :h])),
+           "max_rel_diff_o_vs_single_pass": rel(o_split, ref),
+           "max_rel_diff_state_vs_single_pass": rel(final, lst)}
+    del q3, k3, g3, b3, v3, S03, o3, st3, final, o_split, ref
+    return out
+
+
 class ClockSampler:
     """nvidia-smi clocks/throttle reasons sampled every 200 ms during the timed region."""
 
@@ -446,6 +501,7 @@ def run_ours(args):
                                   "frac": l_ach / lpeak, "alg_bytes_per_launch": lb, "peak_kind": lpeak_kind},
                      "grid": f"{LC['B'] * LC['H']} CTAs (one per head) on the SMs",
                      "timed": "separately, after the headline region, CUDA events per launch"}
+        long_line["split_in_two"] = measure_long_split(kda, LC, lq, lo, lst, stream, reps, l_ms)
         del lq, lo, lst
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
