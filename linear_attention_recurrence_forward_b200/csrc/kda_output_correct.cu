@@ -11,10 +11,13 @@
 // parallelism, which splits a long sequence over devices and passes on only the fixed-size
 // state (channel post on the K3 report (t.iss.one), infrastructure paragraph).
 //
-// For bf16 with dk = dv = 128 the product runs on the tensor core: per CTA one head and 128
-// tokens, C by TMA into a 128-byte-swizzled K-major tile, S_in rounded to bf16 into an
-// MN-major tile, D = C S_in (128 x 128 fp32) in tensor memory, then o_in (TMA) + D rounded to
-// bf16 and stored by TMA.  Other dtypes and head sizes take a CUDA-core kernel in fp32.
+// For bf16 with dk = dv = 128 the product runs on the tensor core.  A CTA takes one head and a run
+// of up to 16 tiles of 128 tokens: S_in rounded to bf16 once into an MN-major tile, then per tile C
+// by TMA into a 128-byte-swizzled K-major tile, D = C S_in (128 x 128 fp32) in tensor memory, and
+// o_in (TMA) + D rounded to bf16 and stored by TMA.  The next tile's C is loaded as soon as the
+// product has read the current one, the next o_in as soon as the store has read its staging tile,
+// so the loads of one tile overlap the work on the previous one.  Other dtypes and head sizes take
+// a CUDA-core kernel in fp32.
 #include <cudaTypedefs.h>
 
 #include "kda_internal.cuh"
@@ -25,9 +28,12 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTok = 128;                 // tokens per CTA (the tensor-core product's M)
+constexpr int kTok = 128;                 // tokens per tile (the tensor-core product's M)
 constexpr int kD = 128;
+constexpr int kTilesPerCta = 16;          // tiles of one head per CTA (S_in converted once for them)
 constexpr int kThreads = 128;             // 4 warps: one TMEM lane quarter each
+constexpr int kLoader = 0;                // issues the C loads and the products
+constexpr int kStorer = 32;               // stores O and loads the next o_in
 constexpr uint32_t OFF_C = 0;             // C tile: 2 atoms of [128 tokens][64 channels] bf16
 constexpr uint32_t OFF_S = 32768;         // S_in bf16, MN-major (K = dk rows), 2 atoms
 constexpr uint32_t OFF_O = 65536;         // o_in, then o_out: 2 atoms of [128 tokens][64 columns]
@@ -37,21 +43,22 @@ constexpr uint32_t ID_CS = idesc_bf16_f32(128, 128, false, true);
 __global__ void __launch_bounds__(kThreads)
 kda_output_correct_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_oi,
                              const __grid_constant__ CUtensorMap tm_oo, const float* S, int H, int ntiles,
-                             int* status, unsigned long long timeout_ns) {
+                             int nsplit, int* status, unsigned long long timeout_ns) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     uint8_t* sm = smem_raw + (((raw_base + 1023u) & ~1023u) - raw_base);
     const uint32_t sb = smem_u32(sm);
-    __shared__ uint64_t bar_ld, bar_mma, bar_drain;
+    __shared__ uint64_t bar_c, bar_o, bar_mma, bar_drain;
     __shared__ uint32_t tmem_base_s;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int tile = blockIdx.x % ntiles;
-    const size_t bh = blockIdx.x / ntiles;
+    const size_t bh = blockIdx.x / nsplit;
     const int b = (int)(bh / H), h = (int)(bh % H);
-    const int t0 = tile * kTok;
+    const int tile0 = (int)(blockIdx.x % nsplit) * kTilesPerCta;
+    const int tile1 = min(tile0 + kTilesPerCta, ntiles);
 
     if (tid == 0) {
-        mbar_init(&bar_ld, 1);
+        mbar_init(&bar_c, 1);
+        mbar_init(&bar_o, 1);
         mbar_init(&bar_mma, 1);
         mbar_init(&bar_drain, 1);
         fence_mbar_init();
@@ -65,14 +72,19 @@ kda_output_correct_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __g
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tbase = tmem_base_s;
-    if (tid == 0) {
-        mbar_arrive_expect_tx(&bar_ld, 4u * 16384u);
+    auto load_c = [&](int tile) {
+        mbar_arrive_expect_tx(&bar_c, 2u * 16384u);
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            tma_load_4d(sm + OFF_C + x * 16384, &tm_c, &bar_ld, 64 * x, h, t0, b);
-            tma_load_4d(sm + OFF_O + x * 16384, &tm_oi, &bar_ld, 64 * x, h, t0, b);
-        }
-    }
+        for (int x = 0; x < 2; ++x) tma_load_4d(sm + OFF_C + x * 16384, &tm_c, &bar_c, 64 * x, h, tile * kTok, b);
+    };
+    auto load_o = [&](int tile) {
+        mbar_arrive_expect_tx(&bar_o, 2u * 16384u);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) tma_load_4d(sm + OFF_O + x * 16384, &tm_oi, &bar_o, 64 * x, h, tile * kTok, b);
+    };
+    int pending_c = -1, pending_o = -1;   // iteration whose load is in flight (loader / storer)
+    if (tid == kLoader) { load_c(tile0); pending_c = 0; }
+    if (tid == kStorer) { load_o(tile0); pending_o = 0; }
     // S_in -> bf16 B operand (row i = dk index, columns = dv): thread i converts row i
     {
         const float4* src = reinterpret_cast<const float4*>(S + (bh * kD + tid) * kD);
@@ -87,62 +99,84 @@ kda_output_correct_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __g
         }
     }
     fence_proxy_async_smem();
-    bool ok = mbar_wait(&bar_ld, 0, timeout_ns);
-    ok = __syncthreads_and(ok) != 0;
-    if (ok && tid == 0) {
+    __syncthreads();
+    bool ok = true;
+    for (int it = 0, tile = tile0; tile < tile1; ++it, ++tile) {
+        const uint32_t par = (uint32_t)(it & 1);
+        // D = C S_in, then the next C into the tile the product has read
+        if (tid == kLoader) {
+            ok = mbar_wait(&bar_c, par, timeout_ns);
+            if (ok) {
+                pending_c = -1;
+                tc_fence_after_sync();
+                issue_mma<8, false, 16384, true, 16384>(tbase, sb + OFF_C, sb + OFF_S, ID_CS, false);
+                mma_commit(&bar_mma);
+            }
+        }
+        ok = __syncthreads_and(ok) != 0;
+        if (!ok) break;
+        ok = mbar_wait(&bar_mma, par, timeout_ns);
+        if (ok && tid == kLoader && tile + 1 < tile1) { load_c(tile + 1); pending_c = it + 1; }
+        if (ok) ok = mbar_wait(&bar_o, par, timeout_ns);
+        if (ok && tid == kStorer) pending_o = -1;
+        ok = __syncthreads_and(ok) != 0;   // block-uniform: the TMEM loads below are warp-collective
+        if (!ok) break;
         tc_fence_after_sync();
-        issue_mma<8, false, 16384, true, 16384>(tbase, sb + OFF_C, sb + OFF_S, ID_CS, false);
-        mma_commit(&bar_mma);
-    }
-    if (ok) ok = mbar_wait(&bar_mma, 0, timeout_ns);
-    ok = __all_sync(0xffffffffu, ok);   // warp-uniform: the TMEM loads below are warp-collective
-    tc_fence_after_sync();
-    if (ok) {
-        // token row r = this thread's TMEM lane: o = o_in + D, 32 columns at a time
-        const int r = 32 * warp + lane;
-        const uint32_t tl = tbase + ((uint32_t)(32 * warp) << 16);
+        {
+            // token row r = this thread's TMEM lane: o = o_in + D, 32 columns at a time
+            const int r = 32 * warp + lane;
+            const uint32_t tl = tbase + ((uint32_t)(32 * warp) << 16);
 #pragma unroll
-        for (int cb = 0; cb < kD; cb += 32) {
-            float d[32];
-            tmem_ld16(tl + cb, d);
-            tmem_ld16(tl + cb + 16, d + 16);
-            tmem_wait_ld();
+            for (int cb = 0; cb < kD; cb += 32) {
+                float d[32];
+                tmem_ld16(tl + cb, d);
+                tmem_ld16(tl + cb + 16, d + 16);
+                tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-                uint8_t* p = sm + OFF_O + sw128_offset(r, cb + j, 16384);
-                const uint4 w = *reinterpret_cast<const uint4*>(p);
-                const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&w);
-                uint32_t out[4];
+                for (int j = 0; j < 32; j += 8) {
+                    uint8_t* p = sm + OFF_O + sw128_offset(r, cb + j, 16384);
+                    const uint4 w = *reinterpret_cast<const uint4*>(p);
+                    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+                    uint32_t out[4];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const float2 f = __bfloat1622float2(o2[m]);
-                    __nv_bfloat162 q = __floats2bfloat162_rn(f.x + d[j + 2 * m], f.y + d[j + 2 * m + 1]);
-                    out[m] = *reinterpret_cast<uint32_t*>(&q);
+                    for (int m = 0; m < 4; ++m) {
+                        const float2 f = __bfloat1622float2(o2[m]);
+                        __nv_bfloat162 q = __floats2bfloat162_rn(f.x + d[j + 2 * m], f.y + d[j + 2 * m + 1]);
+                        out[m] = *reinterpret_cast<uint32_t*>(&q);
+                    }
+                    *reinterpret_cast<uint4*>(p) = make_uint4(out[0], out[1], out[2], out[3]);
                 }
-                *reinterpret_cast<uint4*>(p) = make_uint4(out[0], out[1], out[2], out[3]);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before_sync();   // the next product overwrites D
+        __syncthreads();
+        if (tid == kStorer) {
+            // rows past T are clipped by the tensor map; the next o_in lands once the staging tile is read
+            tma_store_4d(&tm_oo, sm + OFF_O, 0, h, tile * kTok, b);
+            tma_store_4d(&tm_oo, sm + OFF_O + 16384, 64, h, tile * kTok, b);
+            bulk_commit_group();
+            if (tile + 1 < tile1) {
+                bulk_wait_read_all();
+                load_o(tile + 1);
+                pending_o = it + 1;
             }
         }
     }
-    fence_proxy_async_smem();
-    tc_fence_before_sync();
-    ok = __syncthreads_and(ok) != 0;
-    if (tid == 0) {
-        if (ok) {
-            // rows past T are clipped by the tensor map
-            tma_store_4d(&tm_oo, sm + OFF_O, 0, h, t0, b);
-            tma_store_4d(&tm_oo, sm + OFF_O + 16384, 64, h, t0, b);
-            bulk_commit_group();
-            bulk_wait_all();
-        } else {
-            report_status(status, KDA_ERR_TIMEOUT);
-            // nothing of this CTA may still be in flight when it exits
-            mma_commit(&bar_drain);
-            (void)mbar_wait(&bar_drain, 0, timeout_ns);
-            (void)mbar_wait(&bar_ld, 0, timeout_ns);
-        }
+    if (!ok && tid == 0) report_status(status, KDA_ERR_TIMEOUT);
+    // nothing of this CTA may still be in flight when it exits
+    if (tid == kLoader) {
+        mma_commit(&bar_drain);
+        if (!mbar_wait(&bar_drain, 0, timeout_ns)) report_status(status, KDA_ERR_TIMEOUT);
+        if (pending_c >= 0) (void)mbar_wait(&bar_c, (uint32_t)(pending_c & 1), timeout_ns);
     }
-    tc_fence_after_sync();
+    if (tid == kStorer) {
+        bulk_wait_all();
+        if (pending_o >= 0) (void)mbar_wait(&bar_o, (uint32_t)(pending_o & 1), timeout_ns);
+    }
+    tc_fence_before_sync();
     __syncthreads();
+    tc_fence_after_sync();
     if (warp == 0) tmem_dealloc(tbase, kD);
 }
 
@@ -223,8 +257,10 @@ cudaError_t launch_output_correct(const void* C, const float* S, const void* o_i
         if (!make_map128(&mc, C, B, T, H) || !make_map128(&mi, o_in, B, T, H) || !make_map128(&mo, o_out, B, T, H))
             return cudaErrorInvalidValue;
         const int ntiles = (T + kTok - 1) / kTok;
-        const unsigned grid = (unsigned)((size_t)B * H * ntiles);
-        kda_output_correct_tc_kernel<<<grid, kThreads, SMEM_DYN, s>>>(mc, mi, mo, S, H, ntiles, status, timeout_ns);
+        const int nsplit = (ntiles + kTilesPerCta - 1) / kTilesPerCta;
+        const unsigned grid = (unsigned)((size_t)B * H * nsplit);
+        kda_output_correct_tc_kernel<<<grid, kThreads, SMEM_DYN, s>>>(mc, mi, mo, S, H, ntiles, nsplit, status,
+                                                                       timeout_ns);
         return cudaGetLastError();
     }
     if (dtype == KDA_DTYPE_BF16) return launch_simt<__nv_bfloat16>(C, S, o_in, o_out, B, T, H, dk, dv, s);

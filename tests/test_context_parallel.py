@@ -200,6 +200,9 @@ def test_output_correct_rejects_bad_arguments(L):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("dtype,dk,dv,T", [("bf16", 128, 128, 300), ("bf16", 128, 128, 128), ("bf16", 128, 128, 1),
+                                           # 16, 17 and 40 tiles of 128 tokens: one run of tiles per CTA, a
+                                           # second CTA with one tile, three CTAs with a ragged last tile
+                                           ("bf16", 128, 128, 2048), ("bf16", 128, 128, 2049), ("bf16", 128, 128, 5000),
                                            ("bf16", 64, 128, 77), ("fp32", 64, 64, 100), ("fp32", 128, 128, 33)])
 def test_output_correct_kernel_matches_a_cpu_product(dtype, dk, dv, T):
     from linear_attention_recurrence_forward_b200.inputs import torch_dtype
