@@ -858,10 +858,10 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (nchunks > 0 && !convert_gate(0)) ok = false;
             if (nchunks > 1 && !convert_gate(1)) ok = false;
         }
-        // With the prologue every thread of this group reads the chunk's norms, which the prep group
-        // writes before the KQ hand-off: each waits for that hand-off itself.  (The next phase of
-        // bar_kq needs this chunk's MMA3 to have completed, so the parity cannot be a phase ahead.)
-        if (kFused && stid != 0 && nchunks > 0 && ok) ok = mbar_wait(&bar_kq, 0u, p.timeout_ns);
+        // With the prologue this group reads each chunk's norms (Y and O), which the prep group writes
+        // before that chunk's KQ hand-off.  The leader waits for the hand-off (acquire) before it meets
+        // the other threads at the barrier at the top of the chunk's loop iteration, and every read
+        // comes after that barrier, so the norms are visible to all of them.
         for (int chunk = 0; chunk < nchunks; ++chunk) {
             const uint32_t par = chunk & 1;
             const int t0 = chunk * kC;
@@ -1016,7 +1016,6 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 ok = mbar_wait(&bar_kq, par ^ 1u, p.timeout_ns);
                 if (ok) issue_for_chunk(chunk + 1);
             }
-            if (kFused && stid != 0 && chunk + 1 < nchunks && ok) ok = mbar_wait(&bar_kq, par ^ 1u, p.timeout_ns);
             if (gate_warp && chunk + 2 < nchunks && !convert_gate(chunk + 2)) ok = false;
         }
         if (!ok && stid == 0) report_status(p.status, KDA_ERR_TIMEOUT);
