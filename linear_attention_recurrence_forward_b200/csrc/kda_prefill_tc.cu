@@ -65,7 +65,8 @@ constexpr int kThreads = 512;   // 16 warps
 constexpr int kPrepThreads = 256;
 constexpr int kSerialThreads = 256;
 constexpr uint32_t kBarPrep = 1, kBarSerial = 2;   // named hardware barriers
-constexpr int kIssuer = 0;                         // prep thread that issues the g loads (and chunk 0's q, k) and signals
+constexpr int kIssuer = 0;                         // prep thread that issues the g loads (with the prologue chunk 0's
+                                                   // only), chunk 0's q, k, and the hand-off signals
 constexpr int kMma1Issuer = 224;                   // prep thread that issues MMA1 (warp 7: lightest in the solve)
 constexpr int kGateWarp0 = 10, kGateWarps = 6;     // with the prologue: the recurrence warps that convert the gate
 
@@ -76,6 +77,8 @@ constexpr uint32_t OFF_RAW_G = 32768;
 constexpr uint32_t OFF_V = 49152;           // v, then Y = V - Kt S, then U (MN-major B, K = 64 tokens)
 constexpr uint32_t OFF_AP = 65536;          // prep operand region (56 KB)
 constexpr uint32_t OFF_A1 = OFF_AP;                 // [Qt0;Kt0;Qt1;Kt1] block-middle refs, K-major, 2 x 16 KB
+                                                    // (with the prologue, from a chunk's MMA1 to the next chunk's
+                                                    // scan: that next chunk's converted gate, f16 in the g tile's layout)
 constexpr uint32_t OFF_BB = OFF_AP + 32768;         // [Kh0(16);Kh1(48);Kh0(48)], K-major, 96 rows, 2 x 12 KB
 // The solve's scratch, in the MMA1 B-operand space (free once MMA1 is done; the A-operand space is
 // left alone): the diagonal 16x16 blocks of A in fp32 (padded rows of kLdD floats), A in bf16
