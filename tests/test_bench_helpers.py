@@ -1,0 +1,36 @@
+"""bench.py's byte counts and recorded ncu traffic (CPU).
+
+The roofline divides algorithmic bytes per launch by the launch time, so the counts are pinned here
+to figures derived by hand: per token-head, prefill reads q, k, g (dk each), v (dv) and beta and
+writes o (dv), all bf16: 2 * (3 * 128 + 128) + 2 + 2 * 128 = 1282 B at d = 128; per head it reads S0
+and writes S_T, 64 KiB each.  A decode head-step reads and writes the 64 KiB fp32 state and moves
+1026 B of token inputs and 256 B of output.
+"""
+import bench
+
+
+def test_prefill_bytes_of_the_k3_workload():
+    assert bench.prefill_alg_bytes(4, 8192, 96, 128, 128) == 4 * 8192 * 96 * 1282 + 2 * 4 * 96 * 65536
+    assert bench.prefill_alg_bytes(4, 8192, 96, 128, 128) == 4_083_154_944
+    # the long-context workload starts from a zero state: S_T is written, S0 is not read
+    assert bench.prefill_alg_bytes(1, 65536, 96, 128, 128, with_s0=False) == 65536 * 96 * 1282 + 96 * 65536
+
+
+def test_decode_bytes_of_a_step():
+    per_head_step = 2 * 65536 + 1026 + 256
+    assert per_head_step == 132_354
+    assert bench.decode_alg_bytes(256, 96, 128, 128) == 256 * 96 * per_head_step
+
+
+def test_recorded_traffic_is_parsed_and_close_to_the_algorithmic_bytes():
+    # a record counts only while the kernel sources it was captured on are unchanged
+    for tag, alg in (("prefill_tc", bench.prefill_alg_bytes(4, 8192, 96, 128, 128)),
+                     ("decode", bench.decode_alg_bytes(256, 96, 128, 128))):
+        t = bench.recorded_traffic(tag)
+        if t is not None:
+            assert 0.95 * alg <= t <= 1.05 * alg, (tag, t, alg)
+
+
+def test_kernel_source_hash_is_stable_and_short():
+    a, b = bench.kernel_source_sha("prefill_tc"), bench.kernel_source_sha("prefill_tc")
+    assert a == b and len(a) == 16 and a != bench.kernel_source_sha("decode")
