@@ -165,6 +165,78 @@ def measure_long_split(kda, LC, lq, lo, lst, stream, reps, l_ms):
     return out
 
 
+def measure_batching(kda, dev, stream, rank, args):
+    """Continuous batching, the paged / variable-length row: (1) one packed prefill over 64 sequences
+    whose lengths are drawn uniformly from 1..2048 (seeded), H = 96, d = 128, each from its own S0;
+    (2) the decode step with the 256 x 96 states in a pool of 512 slots, the sequences on a random
+    permutation of slots.  CUDA events per launch, the same algorithmic byte counts as the dense
+    workloads (tokens x heads x 1282 B plus 128 KiB of S0/S_T per sequence-head; 132,354 B per
+    head-step)."""
+    import torch
+    from linear_attention_recurrence_forward_b200.inputs import make_prefill_inputs, make_decode_inputs
+
+    H, d, nseq = 96, 128, 64
+    gen = torch.Generator()
+    gen.manual_seed(5000 + rank)
+    lengths = torch.randint(1, 2049, (nseq,), generator=gen)
+    cu = torch.zeros(nseq + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(lengths, 0).to(torch.int32)
+    total = int(cu[-1])
+    q, k, v, g, beta, S0 = make_prefill_inputs(1, total, H, d, d, "bf16", seed=5000 + rank, s0_std=0.02,
+                                               zg_mean=-2.0, device=str(dev))
+    q, k, v, g, beta = (x[0].contiguous() for x in (q, k, v, g, beta))
+    S0n = (torch.randn((nseq, H, d, d), generator=gen) * 0.02).to(dev)
+    cu_d = cu.to(dev)
+    o = torch.empty((total, H, d), dtype=q.dtype, device=dev)
+    ST = torch.empty((nseq, H, d, d), dtype=torch.float32, device=dev)
+    reps = max(3, min(args.steps, 10))
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        torch.cuda.synchronize()
+        for e0, e1 in ev:
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        if kda.kda_get_device_status() != 0:
+            raise RuntimeError("device status after a continuous-batching run")
+        return sum(e0.elapsed_time(e1) for e0, e1 in ev) / reps
+
+    peak, peak_kind = measured_peaks()
+    p_ms = timed(lambda: kda.kda_forward_varlen(q, k, v, g, beta, cu_d, S0n, o=o, S_T=ST, stream=stream))
+    p_bytes = total * H * 1282 + nseq * H * 2 * d * d * 4
+    packed = {"sequences": nseq, "tokens": total, "H": H, "lengths": "uniform on 1..2048 (seeded)",
+              "longest": int(lengths.max()), "launch_ms": p_ms, "tokens_per_s": total / (p_ms / 1e3),
+              "roofline": {"bound": "hbm", "achieved": p_bytes / (p_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                           "frac": p_bytes / (p_ms / 1e3) / 1e9 / peak, "alg_bytes_per_launch": p_bytes,
+                           "peak_kind": peak_kind},
+              "grid": f"{nseq * H} CTAs (one per sequence and head)"}
+    del q, k, v, g, beta, S0, S0n, o, ST
+
+    B, n_slots = 256, 512
+    perm = torch.randperm(n_slots, generator=gen)[:B].to(torch.int32).to(dev)
+    pool = torch.zeros((n_slots, H, d, d), dtype=torch.float32, device=dev)
+    ring = [make_decode_inputs(B, H, d, d, "bf16", gen=None, seed=6000 + i, device=str(dev))[:5] for i in range(4)]
+    step = [0]
+
+    def paged():
+        kda.kda_decode_step_paged(*ring[step[0] % 4], pool, perm, stream=stream)
+        step[0] += 1
+
+    d_ms = timed(paged)
+    d_bytes = decode_alg_bytes(B, H, d, d)
+    paged_line = {"sequences": B, "slots": n_slots, "ms_per_step": d_ms, "states_per_s": B * H / (d_ms / 1e3),
+                  "roofline": {"bound": "hbm", "achieved": d_bytes / (d_ms / 1e3) / 1e9, "peak": peak,
+                               "unit": "GB/s", "frac": d_bytes / (d_ms / 1e3) / 1e9 / peak,
+                               "alg_bytes_per_launch": d_bytes, "peak_kind": peak_kind}}
+    del pool, ring
+    return {"packed_prefill": packed, "paged_decode": paged_line,
+            "timed": "separately, after the headline region, CUDA events per launch"}
+
+
 class ClockSampler:
     """nvidia-smi clocks/throttle reasons sampled every 200 ms during the timed region."""
 
@@ -471,6 +543,9 @@ def run_ours(args):
                               "(an unfused pipeline also reads and writes them once more in a separate pass)"}
         del raw
 
+    # ---- continuous batching: packed prefill of mixed lengths and the paged decode step, timed alone
+    batching_line = None if args.no_batching else measure_batching(kda, dev, stream, rank, args)
+
     # ---- the long-context workload (B1 T65536 H96, S0 = 0, 1024 chunks carried in sequence), timed alone
     long_line = None
     if not args.no_long:
@@ -562,6 +637,7 @@ def run_ours(args):
         "long_context": long_line,
         "state_emission": states_line,
         "fused_prologue": fused_line,
+        "continuous_batching": batching_line,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": 2 * args.steps,
@@ -623,6 +699,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-states", action="store_true", help="skip the state-emission (every 512 tokens) timing")
     ap.add_argument("--no-long", action="store_true", help="skip the long-context (T = 65536) timing")
+    ap.add_argument("--no-batching", action="store_true",
+                    help="skip the continuous-batching timings (packed prefill, paged decode)")
     ap.add_argument("--decode-only", action="store_true",
                     help="profiling: run only decode steps back to back (no prefill between them) and print their "
                          "timing; not the benchmark line")
