@@ -418,7 +418,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
     import linear_attention_recurrence_forward_b200 as kda
-    from linear_attention_recurrence_forward_b200.inputs import make_prefill_inputs, make_decode_inputs
+    from linear_attention_recurrence_forward_b200.inputs import make_prefill_inputs, make_decode_inputs, fingerprint
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -443,6 +443,9 @@ def run_ours(args):
     S = torch.zeros((D["batch"], D["H"], D["dk"], D["dv"]), dtype=torch.float32, device=dev)
     od = torch.empty((D["batch"], D["H"], D["dv"]), dtype=q.dtype, device=dev)
     stream = torch.cuda.current_stream()
+    # the exact input bytes of this rank's workloads (before any timing)
+    inputs_sha256 = {"prefill": fingerprint(q, k, v, g, beta, S0),
+                     "decode_ring": fingerprint(*[t for r in ring for t in r])}
 
     def step(i, ev=None):
         if ev is not None:
@@ -623,7 +626,8 @@ def run_ours(args):
         "config": {"workload": f"{P['name']} prefill + {D['name']} decode step",
                    "B": P["B"], "T": P["T"], "H": P["H"], "dk": P["dk"], "dv": P["dv"],
                    "decode_batch": D["batch"], "l2": "inputs larger than L2 (4.1 GB prefill, 1.6 GB decode state)",
-                   "parallelism": f"replicas x{world} (independent batches, no collective)"},
+                   "parallelism": f"replicas x{world} (independent batches, no collective)",
+                   "inputs_sha256": inputs_sha256},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
                      "traffic": recorded_traffic(impl_tag) if P["name"] == DEFAULT_PREFILL_NAME else None,

@@ -38,6 +38,7 @@ __all__ = [
     "make_decode_inputs",
     "make_prefill_raw_inputs",
     "torch_dtype",
+    "fingerprint",
 ]
 
 
@@ -174,3 +175,22 @@ def make_decode_inputs(batch: int, H: int, dk: int, dv: int, dtype: str = "bf16"
     q, k, v, g, beta, _ = make_prefill_inputs(batch, 1, H, dk, dv, dtype, gen=gen, device=device)
     return (q.view(batch, H, dk), k.view(batch, H, dk), v.view(batch, H, dv),
             g.view(batch, H, dk), beta.view(batch, H))
+
+
+def fingerprint(*tensors) -> str:
+    """SHA-256 (hex) of the exact bytes of the given tensors (None entries skipped), each preceded by
+    its dtype and shape, in the order given: the identity of a run's inputs, whichever side (the
+    library or the oracle) consumes them.  Device tensors are copied to the host in 256 MiB pieces."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for t in tensors:
+        if t is None:
+            continue
+        t = t.contiguous()
+        h.update(f"{t.dtype}:{tuple(t.shape)};".encode())
+        flat = t.view(-1).view(torch.uint8) if t.numel() else t.new_empty(0, dtype=torch.uint8)
+        step = 256 << 20
+        for i in range(0, flat.numel(), step):
+            h.update(flat[i:i + step].cpu().numpy().tobytes())
+    return h.hexdigest()

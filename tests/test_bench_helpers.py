@@ -34,3 +34,13 @@ def test_recorded_traffic_is_parsed_and_close_to_the_algorithmic_bytes():
 def test_kernel_source_hash_is_stable_and_short():
     a, b = bench.kernel_source_sha("prefill_tc"), bench.kernel_source_sha("prefill_tc")
     assert a == b and len(a) == 16 and a != bench.kernel_source_sha("decode")
+
+
+def test_input_fingerprint_identifies_the_seeded_bytes():
+    from linear_attention_recurrence_forward_b200.inputs import make_prefill_inputs, fingerprint
+    a = make_prefill_inputs(1, 130, 2, 64, 64, "bf16", seed=3, s0_std=0.05)
+    b = make_prefill_inputs(1, 130, 2, 64, 64, "bf16", seed=3, s0_std=0.05)
+    c = make_prefill_inputs(1, 130, 2, 64, 64, "bf16", seed=4, s0_std=0.05)
+    assert fingerprint(*a) == fingerprint(*b) and fingerprint(*a) != fingerprint(*c)
+    # the same values in another dtype are other bytes
+    assert fingerprint(a[0]) != fingerprint(a[0].float())
