@@ -447,14 +447,20 @@ def run_ours(args):
     inputs_sha256 = {"prefill": fingerprint(q, k, v, g, beta, S0),
                      "decode_ring": fingerprint(*[t for r in ring for t in r])}
 
+    nvtx = torch.cuda.nvtx   # ranges for profilers (ncu --nvtx); no-ops otherwise
+
     def step(i, ev=None):
         if ev is not None:
             ev[0].record(stream)
+        nvtx.range_push("kda.prefill")
         kda.kda_forward_chunked(q, k, v, g, beta, S0, o=o, S_T=ST, stream=stream)
+        nvtx.range_pop()
         if ev is not None:
             ev[1].record(stream)
         x = ring[i % DECODE_RING]
+        nvtx.range_push("kda.decode")
         kda.kda_decode_step(*x, S, o=od, stream=stream)
+        nvtx.range_pop()
         if ev is not None:
             ev[2].record(stream)
 
