@@ -165,7 +165,7 @@ def measure_long_split(kda, LC, lq, lo, lst, stream, reps, l_ms):
     return out
 
 
-def measure_batching(kda, dev, stream, rank, args):
+def measure_batching(kda, dev, stream, rank, args, H=96, d=128, nseq=64, max_len=2048, batch=256, n_slots=512):
     """Continuous batching, the paged / variable-length row: (1) one packed prefill over 64 sequences
     whose lengths are drawn uniformly from 1..2048 (seeded), H = 96, d = 128, each from its own S0;
     (2) the decode step with the 256 x 96 states in a pool of 512 slots, the sequences on a random
@@ -175,10 +175,9 @@ def measure_batching(kda, dev, stream, rank, args):
     import torch
     from linear_attention_recurrence_forward_b200.inputs import make_prefill_inputs, make_decode_inputs
 
-    H, d, nseq = 96, 128, 64
     gen = torch.Generator()
     gen.manual_seed(5000 + rank)
-    lengths = torch.randint(1, 2049, (nseq,), generator=gen)
+    lengths = torch.randint(1, max_len + 1, (nseq,), generator=gen)
     cu = torch.zeros(nseq + 1, dtype=torch.int32)
     cu[1:] = torch.cumsum(lengths, 0).to(torch.int32)
     total = int(cu[-1])
@@ -207,8 +206,8 @@ def measure_batching(kda, dev, stream, rank, args):
 
     peak, peak_kind = measured_peaks()
     p_ms = timed(lambda: kda.kda_forward_varlen(q, k, v, g, beta, cu_d, S0n, o=o, S_T=ST, stream=stream))
-    p_bytes = total * H * 1282 + nseq * H * 2 * d * d * 4
-    packed = {"sequences": nseq, "tokens": total, "H": H, "lengths": "uniform on 1..2048 (seeded)",
+    p_bytes = total * H * (2 * (3 * d + d) + 2 + 2 * d) + nseq * H * 2 * d * d * 4   # 1282 B per token-head at d = 128
+    packed = {"sequences": nseq, "tokens": total, "H": H, "lengths": f"uniform on 1..{max_len} (seeded)",
               "longest": int(lengths.max()), "launch_ms": p_ms, "tokens_per_s": total / (p_ms / 1e3),
               "roofline": {"bound": "hbm", "achieved": p_bytes / (p_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
                            "frac": p_bytes / (p_ms / 1e3) / 1e9 / peak, "alg_bytes_per_launch": p_bytes,
@@ -216,7 +215,7 @@ def measure_batching(kda, dev, stream, rank, args):
               "grid": f"{nseq * H} CTAs (one per sequence and head)"}
     del q, k, v, g, beta, S0, S0n, o, ST
 
-    B, n_slots = 256, 512
+    B = batch
     perm = torch.randperm(n_slots, generator=gen)[:B].to(torch.int32).to(dev)
     pool = torch.zeros((n_slots, H, d, d), dtype=torch.float32, device=dev)
     ring = [make_decode_inputs(B, H, d, d, "bf16", gen=None, seed=6000 + i, device=str(dev))[:5] for i in range(4)]

@@ -44,3 +44,45 @@ def test_input_fingerprint_identifies_the_seeded_bytes():
     assert fingerprint(*a) == fingerprint(*b) and fingerprint(*a) != fingerprint(*c)
     # the same values in another dtype are other bytes
     assert fingerprint(a[0]) != fingerprint(a[0].float())
+
+
+def test_batching_leg_shapes_and_bytes(monkeypatch):
+    """The continuous-batching leg at tiny sizes on the CPU, with the library and CUDA events stubbed:
+    the packed layout, the slot table and the byte counts it reports."""
+    import types
+    import torch
+
+    class Event:
+        def __init__(self, enable_timing=True):
+            pass
+
+        def record(self, stream=None):
+            pass
+
+        def elapsed_time(self, other):
+            return 2.0
+
+    monkeypatch.setattr(torch.cuda, "Event", Event)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda: None)
+    seen = {}
+
+    def varlen(q, k, v, g, beta, cu, S0, o=None, S_T=None, stream=None):
+        seen["varlen"] = (q.shape, v.shape, beta.shape, cu.dtype, int(cu[-1]), S0.shape, o.shape, S_T.shape)
+
+    def paged(q, k, v, g, beta, pool, slots, stream=None):
+        seen["paged"] = (q.shape, pool.shape, slots.dtype, len(set(slots.tolist())), int(slots.max()))
+
+    kda = types.SimpleNamespace(kda_forward_varlen=varlen, kda_decode_step_paged=paged,
+                                kda_get_device_status=lambda: 0)
+    out = bench.measure_batching(kda, torch.device("cpu"), None, 0, types.SimpleNamespace(steps=3),
+                                 H=2, d=64, nseq=5, max_len=100, batch=6, n_slots=16)
+    tokens = out["packed_prefill"]["tokens"]
+    assert seen["varlen"] == ((tokens, 2, 64), (tokens, 2, 64), (tokens, 2), torch.int32, tokens, (5, 2, 64, 64),
+                              (tokens, 2, 64), (5, 2, 64, 64))
+    # 642 B per token-head at d = 64 (q, k, g, v in and o out in bf16, and beta), 2 x 16 KiB of state per head
+    assert out["packed_prefill"]["roofline"]["alg_bytes_per_launch"] == tokens * 2 * 642 + 5 * 2 * 2 * 64 * 64 * 4
+    assert out["packed_prefill"]["roofline"]["alg_bytes_per_launch"] == bench.prefill_alg_bytes(1, tokens, 2, 64, 64) + \
+        (5 - 1) * 2 * 2 * 64 * 64 * 4
+    assert seen["paged"][:3] == ((6, 2, 64), (16, 2, 64, 64), torch.int32)
+    assert seen["paged"][3] == 6 and seen["paged"][4] < 16            # distinct slots inside the pool
+    assert out["paged_decode"]["roofline"]["alg_bytes_per_launch"] == bench.decode_alg_bytes(6, 2, 64, 64)
