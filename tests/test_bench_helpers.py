@@ -86,3 +86,55 @@ def test_batching_leg_shapes_and_bytes(monkeypatch):
     assert seen["paged"][:3] == ((6, 2, 64), (16, 2, 64, 64), torch.int32)
     assert seen["paged"][3] == 6 and seen["paged"][4] < 16            # distinct slots inside the pool
     assert out["paged_decode"]["roofline"]["alg_bytes_per_launch"] == bench.decode_alg_bytes(6, 2, 64, 64)
+
+
+def test_long_split_leg_stacks_the_three_segment_runs(monkeypatch):
+    """The long-context split leg at tiny sizes on the CPU with the library stubbed: one stacked launch of
+    (first half from 0, second half from 0, second half with v = 0 and S0 = I), then the correction of
+    the second half's outputs with the first half's final state, and the state composition."""
+    import types
+    import torch
+    from linear_attention_recurrence_forward_b200.inputs import make_prefill_inputs
+
+    class Event:
+        def __init__(self, enable_timing=True):
+            pass
+
+        def record(self, stream=None):
+            pass
+
+        def elapsed_time(self, other):
+            return 1.0
+
+    monkeypatch.setattr(torch.cuda, "Event", Event)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda: None)
+    B, T, H, d = 1, 128, 2, 64
+    lq = make_prefill_inputs(B, T, H, d, d, "bf16", seed=1)
+    lo = torch.zeros((B, T, H, d), dtype=torch.bfloat16)
+    lst = torch.ones((B, H, d, d))
+    seen = {}
+
+    def forward(q, k, v, g, beta, S0, o=None, S_T=None, stream=None):
+        h = T // 2
+        assert q.shape == (3 * B, h, H, d) and o.shape == (3 * B, h, H, d) and S_T.shape == (3 * B, H, d, d)
+        assert torch.equal(q[0], lq[0][0, :h]) and torch.equal(q[1], lq[0][0, h:]) and torch.equal(q[2], lq[0][0, h:])
+        assert torch.equal(v[1], lq[2][0, h:]) and not torch.any(v[2])
+        assert not torch.any(S0[:2]) and torch.equal(S0[2], torch.eye(d).expand(H, d, d))
+        o.zero_()
+        S_T.copy_(lst.expand(3 * B, H, d, d))
+        seen["forward"] = seen.get("forward", 0) + 1
+
+    def correct(C, S_in, o_in, out=None, stream=None):
+        seen["correct"] = (C.shape, S_in.shape, out.data_ptr() == o_in.data_ptr())
+
+    def compose(M, S, N, out=None, stream=None):
+        out.copy_(lst)
+        seen["compose"] = (M.shape, S.shape, N.shape)
+
+    kda = types.SimpleNamespace(kda_forward_chunked=forward, kda_output_correct=correct, kda_state_compose=compose,
+                                kda_get_device_status=lambda: 0)
+    LC = dict(B=B, T=T, H=H, dk=d, dv=d)
+    out = bench.measure_long_split(kda, LC, lq, lo, lst, None, 3, 1.0)
+    assert seen["correct"] == ((B, T // 2, H, d), (B, H, d, d), True)
+    assert seen["compose"] == ((B, H, d, d), (B, H, d, d), (B, H, d, d))
+    assert out["ctas"] == 3 * B * H and out["segments"] == 2 and out["max_rel_diff_state_vs_single_pass"] == 0.0
